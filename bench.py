@@ -1,0 +1,409 @@
+#!/usr/bin/env python
+"""Benchmark of the SVDQuant W4A4 linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+                    [--workload qkv]
+
+One step = one ``svdq_linear_forward`` (activation kernel + block-scaled FP4
+GEMM with the fused low-rank branch and bias) over the DiT joint-attention QKV
+projection at 1024x1024 (M = 4608 tokens, K = 3072, N = 9216, r = 32), inputs
+resident in HBM.  L2 is flushed (a 256 MiB write, outside the per-step CUDA
+events) between steps.  Metric: TFLOP/s = 2 M N K / device time per step
+(the low-rank flops 2 M r (K + N) are not counted).
+
+Multi-GPU (torchrun, one rank per GPU): the layer is run as independent
+replicas (token-parallel data parallelism, weights replicated, no collective on
+the data path); value = all ranks' flops / max-over-ranks device time.
+
+``--impl reference`` times the CPU oracle (the only other implementation of the
+method available) on the host cores, on a bounded row sample of the same
+workload, and prints the same JSON line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "SVDQ W4A4 linear TFLOP/s and % of B200 FP4 tensor peak (HBM % at small M)"
+UNIT = "TFLOP/s"
+FP4_SPEC_TFLOPS = 9000.0          # dense NVFP4, NVIDIA B200 datasheet
+FP4_OVER_BF16 = 4.0               # nominal dense ratio fp4 : bf16 (9 / 2.25 PFLOP/s)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+GEMM_SRC = os.path.join(ROOT, "w4a4_rank_corrected_act_b200", "csrc", "fp4_gemm.cuh")
+ACT_SRC = os.path.join(ROOT, "w4a4_rank_corrected_act_b200", "csrc", "act_quant.cuh")
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def _src_sha(path: str) -> str:
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def _profile_traffic(kernel_src: str, name: str):
+    """dram bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source (sha recorded in the summary); else None."""
+    p = os.path.join(ROOT, "profiles", name)
+    if not os.path.exists(p):
+        return None
+    sha = _src_sha(kernel_src)
+    traffic, src = None, None
+    with open(p) as f:
+        for line in f:
+            if line.startswith("source_sha:"):
+                src = line.split(":", 1)[1].strip()
+            if line.startswith("traffic_bytes_per_launch:"):
+                traffic = float(line.split(":", 1)[1].strip())
+    return traffic if src == sha else None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# native (CUDA) arm
+# ---------------------------------------------------------------------------
+
+def run_native(args):
+    import torch
+    import torch.distributed as dist
+
+    import w4a4_rank_corrected_act_b200 as svdq
+    from workloads import gen
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    spec = gen.workload(args.workload)
+    M, K, N, r = spec.M, spec.K, spec.N, spec.r
+    d = gen.make_linear(spec)
+    st = torch.cuda.current_stream()
+    sh = int(st.cuda_stream)
+
+    def dev(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
+
+    lin = svdq.SvdqLinear(dev(d["W"]), torch.from_numpy(d["lam"]).cuda(), dev(d["bias"]), r=r)
+    X = dev(d["X"])
+    Y = torch.empty((M, N), dtype=torch.int16, device="cuda")
+    nb = lin.workspace_bytes(M)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def step():
+        svdq.svdq_linear_forward(X.data_ptr(), M, lin.w, Y.data_ptr(), ws.data_ptr(), nb, sh)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    svdq.svdq_clear_device_status(sh)
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    with ClockSampler(local) as clk:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(st)
+            step()
+            ends[i].record(st)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    status = svdq.svdq_get_device_status(sh)
+    if status:
+        raise SystemExit(f"device status word {status:#x}: a kernel gave up a wait")
+
+    flops = 2.0 * M * N * K
+    value = world * flops * args.steps / (total_ms * 1e-3) / 1e12
+    ms_per_step = total_ms / args.steps
+
+    # dominant kernel alone: the FP4 GEMM (svdq_gemm on the act kernel's output),
+    # and the activation kernel alone, each timed with events on this stream
+    a = svdq.svdq_quantize_act
+    codes_t = torch.empty(svdq.svdq_act_codes_bytes(M, K), dtype=torch.uint8, device="cuda")
+    scales_t = torch.empty(svdq.svdq_act_scales_bytes(M, K), dtype=torch.uint8, device="cuda")
+    d_t = torch.empty((M, max(r, 1)), dtype=torch.int16, device="cuda")
+    codes_p, scales_p, d_p = codes_t.data_ptr(), scales_t.data_ptr(), d_t.data_ptr()
+    reps = max(5, args.steps)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(2 * reps)]
+    for i in range(reps):
+        flush.zero_()
+        ev[i][0].record(st)
+        a(X.data_ptr(), M, lin.w, codes_p, scales_p, d_p, sh)
+        ev[i][1].record(st)
+    for i in range(reps):
+        flush.zero_()
+        ev[reps + i][0].record(st)
+        svdq.svdq_gemm(codes_p, scales_p, d_p, M, lin.w, Y.data_ptr(), sh)
+        ev[reps + i][1].record(st)
+    torch.cuda.synchronize()
+    act_ms = statistics.mean(s.elapsed_time(e) for s, e in ev[:reps])
+    gemm_ms = statistics.mean(s.elapsed_time(e) for s, e in ev[reps:])
+    peaks, peak_kind = _peaks()
+    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+    gemm_tflops = flops / (gemm_ms * 1e-3) / 1e12
+    act_bytes = M * K * 2 + K * 4 + K * r * 2 + M * K // 2 + M * K // 16 + M * r * 2
+    act_gbs = act_bytes / (act_ms * 1e-3) / 1e9
+    roofline = {
+        "kernel": "fp4_gemm_kernel", "bound": "tensor", "achieved": round(gemm_tflops, 1),
+        "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(gemm_tflops / fp4_peak, 4),
+        "traffic": _profile_traffic(GEMM_SRC, f"fp4_gemm_{args.workload}.txt"),
+        "peak_source": f"{peak_kind} bf16 burst {peaks['bf16_tflops']} x nominal fp4:bf16 ratio 4",
+        "frac_of_fp4_spec_9pf": round(gemm_tflops / FP4_SPEC_TFLOPS, 4),
+        "algorithmic_flops_per_launch": flops,
+        "launch_us": round(gemm_ms * 1e3, 2),
+    }
+    act = {"kernel": "act_quant_kernel", "bound": "hbm", "achieved": round(act_gbs, 1),
+           "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(act_gbs / peaks["hbm_gbs"], 4),
+           "algorithmic_bytes_per_launch": act_bytes, "launch_us": round(act_ms * 1e3, 2),
+           "traffic": _profile_traffic(ACT_SRC, f"act_quant_{args.workload}.txt")}
+
+    # end to end through the public API with host buffers (pinned), per step:
+    # H2D of X, the layer, D2H of Y
+    Xh = torch.from_numpy(d["X"].view(np.int16).copy()).pin_memory()
+    Yh = torch.empty((M, N), dtype=torch.int16).pin_memory()
+    Xd = torch.empty((M, K), dtype=torch.int16, device="cuda")
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    for i in range(args.warmup):
+        svdq.svdq_linear_forward_host(Xh.data_ptr(), M, lin.w, Yh.data_ptr(), Xd.data_ptr(),
+                                      Y.data_ptr(), ws.data_ptr(), nb, sh)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        e2e_ev[i][0].record(st)
+        svdq.svdq_linear_forward_host(Xh.data_ptr(), M, lin.w, Yh.data_ptr(), Xd.data_ptr(),
+                                      Y.data_ptr(), ws.data_ptr(), nb, sh)
+        e2e_ev[i][1].record(st)
+    torch.cuda.synchronize()
+    e2e_ms = sum(s.elapsed_time(e) for s, e in e2e_ev)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e = {"value": round(world * flops * args.steps / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
+           "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2,
+           "ms_per_step": round(e2e_ms / args.steps, 4)}
+
+    out = None
+    if rank == 0:
+        out = {
+            "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "nvfp4", "data": "synthetic (seeded DiT-shaped inputs; no checkpoint)",
+            "config": {"workload": f"{spec.name}: DiT joint-attention QKV projection at 1024x1024"
+                                   if spec.name == "qkv" else spec.name,
+                       "M": M, "K": K, "N": N, "r": r, "bias": True,
+                       "l2": "flushed between steps (256 MiB write outside the step events)",
+                       "parallelism": f"replicas x{world} (token-parallel, no collective)"},
+            "pct_fp4_peak": {"of_spec_9000": round(value / FP4_SPEC_TFLOPS, 4),
+                             "of_measured_bf16x4": round(value / fp4_peak, 4)},
+            "us_per_layer": round(ms_per_step * 1e3, 2),
+            "roofline": roofline,
+            "kernels": {"act_quant": act},
+            "e2e": e2e,
+            "gpu_launches": 2 * args.steps,
+            "clocks": clk.summary(),
+        }
+        if args.cpu_baseline:
+            out["cpu_baseline"] = cpu_baseline(spec, d, lin.export(), budget_s=args.cpu_seconds)
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return out
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timings
+# ---------------------------------------------------------------------------
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        n = [i.get("num_threads") for i in info if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def cpu_baseline(spec, d, exp, budget_s=15.0, rows=256):
+    """The oracle's forward (activation quantisation, weight dequantisation,
+    float64 GEMM, low-rank branch) on a row sample of the workload, repeated
+    for about `budget_s` seconds; the weight is the library's exported one."""
+    from oracle import svdq_ref as ref
+    prep = dict(inv_lambda=exp["inv_lambda"], L1=exp["L1"], L2t=exp["L2t"],
+                w_codes=exp["w_codes"], w_scales=exp["w_scales"], bias=d["bias"])
+    X = d["X"][:rows]
+    ref.linear_forward(X[:4], prep)          # warm the BLAS / page in
+    n, t0 = 0, time.perf_counter()
+    while True:
+        ref.linear_forward(X, prep)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or n >= 50:
+            break
+    flops = 2.0 * rows * spec.N * spec.K * n
+    return {"value": flops / el / 1e12, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"{rows} of {spec.M} token rows x {n} repetitions ({el:.1f} s), full K and N; "
+                      "oracle forward incl. per-call weight dequantisation"}
+
+
+def run_reference(args):
+    """The CPU oracle as the reference arm, end to end on the host cores."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return None
+    from oracle import svdq_ref as ref
+    from workloads import gen
+    spec = gen.workload(args.workload)
+    d = gen.make_linear(spec)
+    prep = ref.prepare_weight(d["W"], d["lam"], d["bias"], spec.r)   # offline, untimed
+    rows = args.ref_rows
+    X = d["X"][:rows]
+    for _ in range(args.warmup):
+        ref.linear_forward(X, prep)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        ref.linear_forward(X, prep)
+        times.append(time.perf_counter() - t0)
+    el = sum(times)
+    flops = 2.0 * rows * spec.N * spec.K * args.steps
+    value = flops / el / 1e12
+    out = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded DiT-shaped inputs; no checkpoint)",
+        "config": {"workload": f"{spec.name}: DiT joint-attention QKV projection at 1024x1024"
+                               if spec.name == "qkv" else spec.name,
+                   "M": spec.M, "K": spec.K, "N": spec.N, "r": spec.r,
+                   "parallelism": "host cores (CPU oracle)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+                         "sample": f"{rows} of {spec.M} token rows per step, full K and N"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(out), flush=True)
+    return out
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", default="qkv")
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-rows", type=int, default=128)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1 and int(os.environ.get("RANK", "0")) != 0:
+        args.cpu_baseline = False
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        raise SystemExit("for --gpus > 1 launch with torch.distributed.run (one rank per GPU)")
+    return run_native(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,213 @@
+/*
+ * svdq.h -- C ABI of the B200 (sm_100a) SVDQuant W4A4 linear layer.
+ *
+ * The layer computes
+ *     Y = Xhat L1 L2 + Q4(Xhat) Q4(R)^T + b,   Xhat = X diag(1/lambda),
+ *     R = W diag(lambda) - (L1 L2)^T,
+ * where W (N x K, nn.Linear layout) is split offline into a rank-r bf16 branch
+ * L1 (K x r), L2 (r x N) and a residual R quantised to NVFP4 (E2M1 codes, one
+ * E4M3 scale per 16 consecutive elements along K).  Activations are quantised
+ * to NVFP4 on every call; the bulk of the work runs as a 4-bit x 4-bit
+ * block-scaled GEMM on the tensor cores and the low-rank correction in 16 bit.
+ *
+ * Sources of the operation (web pages on SVDQuant / Nunchaku):
+ *   - W4A4, activation outliers migrated into the weights, the hard part as a
+ *     16-bit low-rank branch and the rest in 4 bit: aiphreaks.com "Bringing
+ *     Nunchaku 4-bit Diffusion Inference to Diffusers", section "Technical
+ *     Breakdown and Performance Metrics"; chaosnode.de "Nunchaku Lite: 4-Bit
+ *     Diffusion-Inferenz direkt in Diffusers", section "Die Technik: SVDQuant".
+ *   - low-rank component plus residual, most work in 4-bit tensor cores and
+ *     the correction in higher precision: imaginepro.ai "Nunchaku 4-Bit
+ *     Diffusion Inference in Diffusers: A Practical Guide", section "Under
+ *     the Hood: 4-Bit Quantization for Diffusion Models".
+ *   - NVFP4 on Blackwell / B200: chaosnode.de, section "Hardware-Support";
+ *     rank 32: watch-ia.com checkpoint name "...nunchaku-lite-nvfp4_r32...".
+ *   - drop-in replacement of a linear layer (patched nn.Linear), offline
+ *     quantisation separate from inference: chaosnode.de, section "Nunchaku
+ *     Lite vs. Original"; watch-ia.com (diffuse-compressor four-step flow).
+ *
+ * Conventions (all entry points):
+ *   - Tensors are row-major.  bf16 values are passed as uint16_t bit patterns.
+ *   - "device" pointers must be CUDA device memory on the device that is
+ *     current for the calling thread; they must be 16-byte aligned
+ *     (SVDQ_ERR_MISALIGNED otherwise).  The caller owns every buffer.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Compute calls are asynchronous on it and never synchronise,
+ *     except where stated (export, device status).
+ *   - Shape limits of the GPU path: K % 256 == 0, N % 128 == 0, r % 8 == 0,
+ *     0 <= r <= 64 and r <= min(N, K) (SVDQ_ERR_UNSUPPORTED_SHAPE otherwise);
+ *     K % 16 != 0, N <= 0, K <= 0 or M < 0 is SVDQ_ERR_INVALID_ARG.  M == 0
+ *     is a valid empty call that does nothing.  M, N, K < 2^31.
+ *   - Errors are returned as status codes; nothing is thrown across the ABI.
+ *     A CUDA launch/runtime failure is SVDQ_ERR_CUDA (its text is kept in a
+ *     thread-local string, see svdq_last_error_detail).
+ *   - The library is stateless apart from a per-device status word that
+ *     kernels set when a bounded wait times out (svdq_get_device_status).
+ */
+#ifndef SVDQ_H_
+#define SVDQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum svdq_status {
+  SVDQ_OK = 0,
+  SVDQ_ERR_INVALID_ARG = 1,        /* null pointer, negative or non-multiple-of-16 size */
+  SVDQ_ERR_UNSUPPORTED_SHAPE = 2,  /* valid layer, but outside the GPU path's limits   */
+  SVDQ_ERR_MISALIGNED = 3,         /* a device pointer is not 16-byte aligned           */
+  SVDQ_ERR_WORKSPACE_TOO_SMALL = 4,
+  SVDQ_ERR_CUDA = 5,               /* CUDA runtime / launch error                       */
+  SVDQ_ERR_TIMEOUT = 6,            /* a kernel's bounded wait expired (device status)   */
+  SVDQ_ERR_SOLVER = 7              /* the eigen-solver of svdq_prepare_weight failed    */
+} svdq_status;
+
+/*
+ * A prepared layer.  All pointers are device pointers owned by the caller
+ * (svdq_weight_bind carves them out of one buffer).  Layouts:
+ *   w_codes    N x K/2 bytes: NVFP4 codes of R, row n holds R[n, :], element
+ *              2j in the low nibble of byte j (E2M1: bit 3 sign, bits 0-2
+ *              magnitude index into {0,.5,1,1.5,2,3,4,6}).
+ *   w_scales   E4M3 scale codes of R in the scale-factor tile layout used by
+ *              the block-scaled tensor-core MMA: 512-byte tiles of 128 rows x
+ *              4 scales (64 K-elements); tile (rb, kb) at byte
+ *              (rb * K/64 + kb) * 512, and inside a tile, row i and scale j at
+ *              (i % 32) * 16 + (i / 32) * 4 + j.  Size N * K / 16 bytes.
+ *   L1         K x r bf16, L1 = U_r diag(sigma_r) of the smoothed weight.
+ *   L2t        N x r bf16, L2^T = V_r.
+ *   inv_lambda K float32, f32(1 / lambda).
+ *   bias       N bf16, or NULL when has_bias == 0.
+ */
+typedef struct svdq_weight {
+  int32_t N, K, r;
+  int32_t has_bias;
+  uint8_t* w_codes;
+  uint8_t* w_scales;
+  uint16_t* L1;
+  uint16_t* L2t;
+  float* inv_lambda;
+  uint16_t* bias;
+} svdq_weight;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* svdq_status_string(svdq_status s);
+
+/* Text of the last SVDQ_ERR_CUDA / SVDQ_ERR_SOLVER seen on this host thread. */
+const char* svdq_last_error_detail(void);
+
+/* Library version, e.g. "svdq-b200 0.1". */
+const char* svdq_version(void);
+
+/* ---------------------------------------------------------------------------
+ * Sizes.  Pure host functions; 0 means the shape is invalid or unsupported.
+ * ------------------------------------------------------------------------- */
+
+/* Bytes of one svdq_weight buffer (all fields, each 256-byte aligned). */
+size_t svdq_weight_bytes(int N, int K, int r, int has_bias);
+
+/* Bytes of activation codes (M x K/2), scales (M rounded up to 128 rows, in
+ * the scale-factor tile layout above) and D (M x r bf16). */
+size_t svdq_act_codes_bytes(int M, int K);
+size_t svdq_act_scales_bytes(int M, int K);
+
+/* Workspace of svdq_linear_forward: codes + scales + D, 256-byte aligned. */
+size_t svdq_forward_workspace_bytes(int M, int N, int K, int r);
+
+/* Workspace of svdq_prepare_weight.  This asks the eigen-solver for its
+ * buffer size and therefore needs a CUDA device (returns 0 without one). */
+size_t svdq_prepare_workspace_bytes(int N, int K, int r);
+
+/* Carve a caller-allocated device buffer of svdq_weight_bytes() bytes into the
+ * fields of *out (pointer arithmetic only, no device access). */
+svdq_status svdq_weight_bind(void* buf, size_t bytes, int N, int K, int r, int has_bias,
+                             svdq_weight* out);
+
+/* ---------------------------------------------------------------------------
+ * Offline preparation (smoothing, rank-r split, residual NVFP4 pack).
+ *   W       device, N x K bf16 (nn.Linear weight)
+ *   lambda  device, K float32 smoothing factors (> 0, finite), calibrated by
+ *           the caller from activation statistics
+ *   bias    device, N bf16, or NULL (must be non-NULL iff w->has_bias)
+ *   w       weight bound with svdq_weight_bind for the same N, K, r
+ *   ws      device workspace of svdq_prepare_workspace_bytes() bytes
+ * Steps: What = f32(W * lambda) per column; L1 = U_r diag(sigma_r),
+ * L2 = V_r^T from the top-r eigenpairs of the float64 Gram matrix of What
+ * (the smaller of What What^T and What^T What), each pair sign-normalised so
+ * the largest-|.| entry of u_i is positive, stored as bf16 (RNE);
+ * R = f32(What - (bf16 L1 bf16 L2)^T) summed in float64; R quantised to NVFP4
+ * along K.  Offline: it creates (and destroys) one cuSOLVER handle per call,
+ * whose own small allocation is the one exception to "never allocates", and
+ * the solver may synchronise the stream.
+ * ------------------------------------------------------------------------- */
+svdq_status svdq_prepare_weight(const uint16_t* W, const float* lambda, const uint16_t* bias,
+                                const svdq_weight* w, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Activation kernel (one HBM pass over X).
+ *   X        device, M x K bf16
+ *   x_codes  device, M x K/2 NVFP4 codes of Xhat = f32(X * inv_lambda)
+ *   x_scales device, svdq_act_scales_bytes(M, K) bytes, tile layout; rows
+ *            M .. roundup(M,128)-1 are written as zero
+ *   D        device, M x r bf16, D = bf16(sum_k bf16(Xhat)_mk bf16(L1)_kj)
+ *            with float32 accumulation; may be NULL when r == 0
+ * ------------------------------------------------------------------------- */
+svdq_status svdq_quantize_act(const uint16_t* X, int M, const svdq_weight* w, uint8_t* x_codes,
+                              uint8_t* x_scales, uint16_t* D, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Block-scaled FP4 GEMM with the low-rank branch and bias fused:
+ *   Y = bf16(deq(x_codes, x_scales) deq(w_codes, w_scales)^T + D L2 + bias),
+ * float32 accumulation in tensor memory.  Inputs as produced by
+ * svdq_quantize_act; Y device, M x N bf16.  Output tiles are 128 x 256 when
+ * N % 256 == 0 and there are at least as many of them as SMs, else 128 x 128;
+ * the environment variable SVDQ_GEMM_BN=128|256 overrides that choice.
+ * ------------------------------------------------------------------------- */
+svdq_status svdq_gemm(const uint8_t* x_codes, const uint8_t* x_scales, const uint16_t* D, int M,
+                      const svdq_weight* w, uint16_t* Y, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Whole layer: svdq_quantize_act then svdq_gemm on `stream`, with the
+ * activation codes, scales and D placed in the caller's workspace `ws`
+ * (svdq_forward_workspace_bytes(M, N, K, r) bytes, device).
+ * ------------------------------------------------------------------------- */
+svdq_status svdq_linear_forward(const uint16_t* X, int M, const svdq_weight* w, uint16_t* Y,
+                                void* ws, size_t ws_bytes, void* stream);
+
+/* Same as svdq_linear_forward but with X and Y in pinned HOST memory: copies
+ * X_host -> X_dev (M x K bf16), runs the layer into Y_dev, copies Y_dev ->
+ * Y_host (M x N bf16), all asynchronously on `stream` (the caller
+ * synchronises before reading Y_host). */
+svdq_status svdq_linear_forward_host(const uint16_t* X_host, int M, const svdq_weight* w,
+                                     uint16_t* Y_host, uint16_t* X_dev, uint16_t* Y_dev,
+                                     void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Test / checkpoint path: copy a prepared weight to host buffers in logical
+ * layouts (codes N x K/2, scales N x K/16 row-major, L1 K x r, L2t N x r,
+ * inv_lambda K).  Any host pointer may be NULL to skip that field.
+ * Synchronises `stream`.
+ * ------------------------------------------------------------------------- */
+svdq_status svdq_weight_export(const svdq_weight* w, uint8_t* host_codes, uint8_t* host_scales,
+                               uint16_t* host_L1, uint16_t* host_L2t, float* host_inv_lambda,
+                               void* stream);
+
+/* Host-only layout conversions between logical [rows][K/16] scales and the
+ * tile layout (rows of the tile layout are `rows` rounded up to 128; padding
+ * entries are written as 0 by to_native and ignored by to_logical). */
+svdq_status svdq_scales_to_logical(const uint8_t* native, int rows, int K, uint8_t* logical);
+svdq_status svdq_scales_to_native(const uint8_t* logical, int rows, int K, uint8_t* native);
+
+/* Synchronise `stream` and report the device status word of the current
+ * device: SVDQ_OK, or SVDQ_ERR_TIMEOUT if a kernel gave up a bounded wait
+ * since the last clear.  *detail (optional) receives the raw word. */
+svdq_status svdq_get_device_status(void* stream, uint32_t* detail);
+svdq_status svdq_clear_device_status(void* stream);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* SVDQ_H_ */

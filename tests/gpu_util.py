@@ -1,0 +1,79 @@
+"""Helpers shared by the GPU tests: device buffers from torch, calls through the
+C ABI binding, and comparisons with the oracle's tolerances."""
+from __future__ import annotations
+
+import numpy as np
+
+from oracle import svdq_ref as ref
+
+
+def torch():
+    import torch as _t
+    return _t
+
+
+def dev_u16(a: np.ndarray):
+    t = torch()
+    return t.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
+
+
+def dev_f32(a: np.ndarray):
+    t = torch()
+    return t.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).cuda()
+
+
+def dev_u8(a: np.ndarray):
+    t = torch()
+    return t.from_numpy(np.ascontiguousarray(a, dtype=np.uint8)).cuda()
+
+
+def to_np_u16(t) -> np.ndarray:
+    return t.cpu().numpy().view(np.uint16)
+
+
+def empty_u8(n: int):
+    t = torch()
+    return t.empty(max(int(n), 256), dtype=t.uint8, device="cuda")
+
+
+def stream() -> int:
+    return int(torch().cuda.current_stream().cuda_stream)
+
+
+def bf16_ulp(x: np.ndarray) -> np.ndarray:
+    """Spacing of bf16 at |x| (8 significant bits), 2^-133 minimum."""
+    a = np.abs(np.asarray(x, dtype=np.float64))
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    return np.where(a > 0, np.maximum(2.0 ** (e - 7), 2.0 ** -133), 2.0 ** -133)
+
+
+def check_y(y_gpu_bits: np.ndarray, y_oracle64: np.ndarray, what: str = "Y"):
+    """Output bar: max|Y_gpu - Y_oracle| <= 4e-3 rms(Y_oracle), and no element off
+    by more than 2 bf16 ulps plus that bound."""
+    yg = ref.bf16_to_f64(y_gpu_bits)
+    yo = ref.bf16_to_f64(ref.f64_to_bf16(y_oracle64))
+    rms = float(np.sqrt(np.mean(y_oracle64 ** 2)))
+    err = np.abs(yg - yo)
+    bound = 4e-3 * rms
+    assert np.all(np.isfinite(yg)), f"{what}: non-finite output"
+    worst = float(err.max()) if err.size else 0.0
+    assert worst <= bound + 2 * float(bf16_ulp(yo).max() if yo.size else 0), \
+        f"{what}: max err {worst:.3e} > bound {bound:.3e}"
+    over = err > bound + 2 * bf16_ulp(yo)
+    assert not np.any(over), f"{what}: {int(over.sum())} elements beyond 2 ulp + 4e-3 rms"
+    return worst / max(rms, 1e-30)
+
+
+def check_d(d_gpu_bits: np.ndarray, d_oracle_bits: np.ndarray, d_abs: np.ndarray):
+    """D bar: |D_gpu - D_oracle| <= 1 bf16 ulp(D_oracle) + 2^-14 sum_k |Xhat_mk L1_kj|.
+
+    The oracle sums the bf16 x bf16 products in f64 and rounds once; the GPU
+    accumulates the same (exact) products in float32: each of 4 partial sums
+    takes K/64 tensor-core accumulation steps, each rounding (or truncating) at
+    most 2^-23 of a partial bounded by the absolute sum, so the error stays
+    below (K/64 + 4) 2^-23 sum|.| <= 2^-14 sum|.| for K <= 16384."""
+    g = ref.bf16_to_f64(d_gpu_bits)
+    o = ref.bf16_to_f64(d_oracle_bits)
+    bound = bf16_ulp(o) + 2.0 ** -14 * d_abs
+    err = np.abs(g - o)
+    assert np.all(err <= bound), f"D: {int((err > bound).sum())} elements off, max {err.max():.3e}"

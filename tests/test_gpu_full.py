@@ -1,0 +1,69 @@
+"""Full-size parity of the CUDA path (the workloads' own shapes), on outputs the
+oracle computes row by row: sampled token rows of the activation codes, scales,
+D and Y, and sampled weight rows of the residual codes and scales (every
+row of those is independent of the others, so a sample is checked exactly)."""
+import numpy as np
+import pytest
+
+import w4a4_rank_corrected_act_b200 as svdq
+from oracle import svdq_ref as ref
+from workloads import gen
+
+from gpu_util import check_d, check_y, dev_f32, dev_u16, empty_u8, stream, to_np_u16, torch
+
+pytestmark = pytest.mark.gpu
+
+FULL = ["qkv", "mlp_up", "mlp_down", "small_m", "block_b1_out"]
+
+
+def _sample(n, k, seed):
+    rng = np.random.default_rng(seed)
+    s = set(rng.choice(n, size=min(k, n), replace=False).tolist())
+    s.update([0, n - 1])
+    return np.array(sorted(s))
+
+
+@pytest.mark.parametrize("name", FULL + ["block_b4_down"])
+def test_full_size_sampled(name):
+    t = torch()
+    spec = gen.workload(name)
+    d = gen.make_linear(spec)
+    M, K, N, r = spec.M, spec.K, spec.N, spec.r
+    lin = svdq.SvdqLinear(dev_u16(d["W"]), dev_f32(d["lam"]), dev_u16(d["bias"]), r=r)
+    exp = lin.export()
+    inv = ref.inv_lambda_of(d["lam"])
+    assert np.array_equal(exp["inv_lambda"].view(np.uint32), inv.view(np.uint32))
+    # weight rows: residual codes/scales given the exported bf16 factors
+    wrows = _sample(N, 96, 1)
+    w_hat = ref.smooth_weight(d["W"][wrows], d["lam"])
+    L2s = np.ascontiguousarray(exp["L2t"][wrows].T)
+    _, wc, ws = ref.residual_quantize(w_hat, exp["L1"], L2s)
+    assert int((wc != exp["w_codes"][wrows]).sum()) == 0
+    assert np.array_equal(ws, exp["w_scales"][wrows])
+    # activations through svdq_quantize_act, then Y through svdq_linear_forward
+    X = dev_u16(d["X"])
+    codes = empty_u8(svdq.svdq_act_codes_bytes(M, K))
+    scales = empty_u8(svdq.svdq_act_scales_bytes(M, K))
+    D = t.empty((M, r), dtype=t.int16, device="cuda")
+    svdq.svdq_quantize_act(X.data_ptr(), M, lin.w, codes.data_ptr(), scales.data_ptr(),
+                           D.data_ptr(), stream())
+    Y = lin.forward(X.view(t.bfloat16))
+    t.cuda.synchronize()
+    rows = _sample(M, 64, 2)
+    xo = ref.quantize_act(d["X"][rows], inv, exp["L1"])
+    cg = codes[: M * K // 2].cpu().numpy().reshape(M, K // 2)[rows]
+    assert int((cg != xo["x_codes"]).sum()) == 0
+    sn = scales.cpu().numpy()
+    logical = np.empty((M, K // 16), np.uint8)
+    svdq.svdq_scales_to_logical(sn.ctypes.data, M, K, logical.ctypes.data)
+    assert np.array_equal(logical[rows], xo["x_scales"])
+    check_d(D.cpu().numpy().view(np.uint16)[rows], xo["D"], xo["D_abs"])
+    # Y rows: the oracle on the exported weight (all weight rows needed here)
+    full_hat = ref.smooth_weight(d["W"], d["lam"])
+    prep = dict(inv_lambda=inv, L1=exp["L1"], L2t=exp["L2t"], w_codes=exp["w_codes"],
+                w_scales=exp["w_scales"], bias=d["bias"])
+    del full_hat
+    o = ref.linear_forward(d["X"], prep, rows=rows)
+    rel = check_y(to_np_u16(Y.view(t.int16))[rows], o["Y64"], name)
+    print(f"{name}: max |dY| / rms = {rel:.2e}")
+    assert svdq.svdq_get_device_status(stream()) == 0

@@ -1,0 +1,260 @@
+"""ctypes binding of the C ABI in include/svdq.h (argument marshalling only).
+
+Every function here has the name of the C entry point it calls and forwards
+plain integers (device / host addresses, sizes, the CUDA stream handle).  No
+step of the layer runs in Python: if the shared library is missing or cannot be
+loaded, every call raises -- there is no fallback.
+
+`SvdqLinear` is a small convenience owner of one prepared layer whose device
+memory comes from PyTorch (PyTorch is used for memory and streams only).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+_PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG_DIR, "libsvdq_b200.so")
+
+SVDQ_OK = 0
+STATUS_NAMES = {
+    0: "SVDQ_OK", 1: "SVDQ_ERR_INVALID_ARG", 2: "SVDQ_ERR_UNSUPPORTED_SHAPE",
+    3: "SVDQ_ERR_MISALIGNED", 4: "SVDQ_ERR_WORKSPACE_TOO_SMALL", 5: "SVDQ_ERR_CUDA",
+    6: "SVDQ_ERR_TIMEOUT", 7: "SVDQ_ERR_SOLVER",
+}
+
+# exported symbols, with (restype, argtypes)
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_SZ = ctypes.c_size_t
+
+
+class svdq_weight(ctypes.Structure):
+    _fields_ = [
+        ("N", ctypes.c_int32), ("K", ctypes.c_int32), ("r", ctypes.c_int32),
+        ("has_bias", ctypes.c_int32),
+        ("w_codes", _P), ("w_scales", _P), ("L1", _P), ("L2t", _P),
+        ("inv_lambda", _P), ("bias", _P),
+    ]
+
+
+_WP = ctypes.POINTER(svdq_weight)
+
+SIGNATURES = {
+    "svdq_status_string": (ctypes.c_char_p, [_I]),
+    "svdq_last_error_detail": (ctypes.c_char_p, []),
+    "svdq_version": (ctypes.c_char_p, []),
+    "svdq_weight_bytes": (_SZ, [_I, _I, _I, _I]),
+    "svdq_act_codes_bytes": (_SZ, [_I, _I]),
+    "svdq_act_scales_bytes": (_SZ, [_I, _I]),
+    "svdq_forward_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
+    "svdq_prepare_workspace_bytes": (_SZ, [_I, _I, _I]),
+    "svdq_weight_bind": (_I, [_P, _SZ, _I, _I, _I, _I, _WP]),
+    "svdq_prepare_weight": (_I, [_P, _P, _P, _WP, _P, _SZ, _P]),
+    "svdq_quantize_act": (_I, [_P, _I, _WP, _P, _P, _P, _P]),
+    "svdq_gemm": (_I, [_P, _P, _P, _I, _WP, _P, _P]),
+    "svdq_linear_forward": (_I, [_P, _I, _WP, _P, _P, _SZ, _P]),
+    "svdq_linear_forward_host": (_I, [_P, _I, _WP, _P, _P, _P, _P, _SZ, _P]),
+    "svdq_weight_export": (_I, [_WP, _P, _P, _P, _P, _P, _P]),
+    "svdq_scales_to_logical": (_I, [_P, _I, _I, _P]),
+    "svdq_scales_to_native": (_I, [_P, _I, _I, _P]),
+    "svdq_get_device_status": (_I, [_P, ctypes.POINTER(ctypes.c_uint32)]),
+    "svdq_clear_device_status": (_I, [_P]),
+}
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+class SvdqError(RuntimeError):
+    def __init__(self, fn: str, status: int, detail: str = ""):
+        self.status = status
+        msg = f"{fn} -> {STATUS_NAMES.get(status, status)}"
+        if detail:
+            msg += f": {detail}"
+        super().__init__(msg)
+
+
+def lib() -> ctypes.CDLL:
+    """Load libsvdq_b200.so (built by ``w4a4_rank_corrected_act_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m w4a4_rank_corrected_act_b200.build`")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(handle, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def _check(fn: str, status: int) -> None:
+    if status != SVDQ_OK:
+        detail = lib().svdq_last_error_detail().decode(errors="replace")
+        raise SvdqError(fn, status, detail if status in (5, 7) else "")
+
+
+def _call(fn: str, *args) -> None:
+    _check(fn, getattr(lib(), fn)(*args))
+
+
+# --------------------------------------------------------------------------
+# one wrapper per entry point (same names as the C ABI)
+# --------------------------------------------------------------------------
+
+def svdq_status_string(s: int) -> str:
+    return lib().svdq_status_string(s).decode()
+
+
+def svdq_version() -> str:
+    return lib().svdq_version().decode()
+
+
+def svdq_weight_bytes(N: int, K: int, r: int, has_bias: int) -> int:
+    return lib().svdq_weight_bytes(N, K, r, has_bias)
+
+
+def svdq_act_codes_bytes(M: int, K: int) -> int:
+    return lib().svdq_act_codes_bytes(M, K)
+
+
+def svdq_act_scales_bytes(M: int, K: int) -> int:
+    return lib().svdq_act_scales_bytes(M, K)
+
+
+def svdq_forward_workspace_bytes(M: int, N: int, K: int, r: int) -> int:
+    return lib().svdq_forward_workspace_bytes(M, N, K, r)
+
+
+def svdq_prepare_workspace_bytes(N: int, K: int, r: int) -> int:
+    return lib().svdq_prepare_workspace_bytes(N, K, r)
+
+
+def svdq_weight_bind(buf: int, nbytes: int, N: int, K: int, r: int, has_bias: int) -> svdq_weight:
+    w = svdq_weight()
+    _call("svdq_weight_bind", buf, nbytes, N, K, r, has_bias, ctypes.byref(w))
+    return w
+
+
+def svdq_prepare_weight(W: int, lam: int, bias: int, w: svdq_weight, ws: int, ws_bytes: int,
+                        stream: int) -> None:
+    _call("svdq_prepare_weight", W, lam, bias or None, ctypes.byref(w), ws, ws_bytes, stream or None)
+
+
+def svdq_quantize_act(X: int, M: int, w: svdq_weight, x_codes: int, x_scales: int, D: int,
+                      stream: int) -> None:
+    _call("svdq_quantize_act", X, M, ctypes.byref(w), x_codes, x_scales, D or None, stream or None)
+
+
+def svdq_gemm(x_codes: int, x_scales: int, D: int, M: int, w: svdq_weight, Y: int,
+              stream: int) -> None:
+    _call("svdq_gemm", x_codes, x_scales, D or None, M, ctypes.byref(w), Y, stream or None)
+
+
+def svdq_linear_forward(X: int, M: int, w: svdq_weight, Y: int, ws: int, ws_bytes: int,
+                        stream: int) -> None:
+    _call("svdq_linear_forward", X, M, ctypes.byref(w), Y, ws, ws_bytes, stream or None)
+
+
+def svdq_linear_forward_host(X_host: int, M: int, w: svdq_weight, Y_host: int, X_dev: int,
+                             Y_dev: int, ws: int, ws_bytes: int, stream: int) -> None:
+    _call("svdq_linear_forward_host", X_host, M, ctypes.byref(w), Y_host, X_dev, Y_dev, ws,
+          ws_bytes, stream or None)
+
+
+def svdq_weight_export(w: svdq_weight, host_codes: int, host_scales: int, host_L1: int,
+                       host_L2t: int, host_inv_lambda: int, stream: int) -> None:
+    _call("svdq_weight_export", ctypes.byref(w), host_codes or None, host_scales or None,
+          host_L1 or None, host_L2t or None, host_inv_lambda or None, stream or None)
+
+
+def svdq_scales_to_logical(native: int, rows: int, K: int, logical: int) -> None:
+    _call("svdq_scales_to_logical", native, rows, K, logical)
+
+
+def svdq_scales_to_native(logical: int, rows: int, K: int, native: int) -> None:
+    _call("svdq_scales_to_native", logical, rows, K, native)
+
+
+def svdq_get_device_status(stream: int = 0) -> int:
+    """Returns the raw device status word (0 = no kernel gave up a wait)."""
+    detail = ctypes.c_uint32(0)
+    st = lib().svdq_get_device_status(stream or None, ctypes.byref(detail))
+    if st not in (SVDQ_OK, 6):
+        _check("svdq_get_device_status", st)
+    return int(detail.value)
+
+
+def svdq_clear_device_status(stream: int = 0) -> None:
+    _call("svdq_clear_device_status", stream or None)
+
+
+# --------------------------------------------------------------------------
+# convenience owner of one prepared layer (device memory from torch)
+# --------------------------------------------------------------------------
+
+def _stream_handle(stream=None) -> int:
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+class SvdqLinear:
+    """A prepared SVDQuant W4A4 linear on the current CUDA device.
+
+    ``W`` (N x K), ``lam`` (K, float32) and ``bias`` (N or None) are device
+    tensors; the weight is prepared once with ``svdq_prepare_weight`` and kept
+    in one torch-allocated buffer bound with ``svdq_weight_bind``.
+    """
+
+    def __init__(self, W, lam, bias=None, r: int = 32, stream=None):
+        import torch
+        N, K = W.shape
+        self.N, self.K, self.r = int(N), int(K), int(r)
+        self.has_bias = bias is not None
+        nbytes = svdq_weight_bytes(self.N, self.K, self.r, int(self.has_bias))
+        if nbytes == 0:
+            raise SvdqError("svdq_weight_bytes", 2, f"N={N} K={K} r={r}")
+        self.buf = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
+        self.w = svdq_weight_bind(self.buf.data_ptr(), nbytes, self.N, self.K, self.r,
+                                  int(self.has_bias))
+        ws_bytes = svdq_prepare_workspace_bytes(self.N, self.K, self.r)
+        ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=W.device)
+        Wc = W.contiguous()
+        lc = lam.contiguous()
+        bc = bias.contiguous() if bias is not None else None
+        svdq_prepare_weight(Wc.data_ptr(), lc.data_ptr(), bc.data_ptr() if bc is not None else 0,
+                            self.w, ws.data_ptr(), ws_bytes, _stream_handle(stream))
+        torch.cuda.current_stream().synchronize() if stream is None else stream.synchronize()
+        del ws
+
+    def workspace_bytes(self, M: int) -> int:
+        return svdq_forward_workspace_bytes(M, self.N, self.K, self.r)
+
+    def forward(self, X, Y=None, ws=None, stream=None):
+        import torch
+        M = X.shape[0]
+        if Y is None:
+            Y = torch.empty((M, self.N), dtype=torch.bfloat16, device=X.device)
+        nb = self.workspace_bytes(M)
+        if ws is None:
+            ws = torch.empty(max(nb, 256), dtype=torch.uint8, device=X.device)
+        svdq_linear_forward(X.data_ptr(), M, self.w, Y.data_ptr(), ws.data_ptr(), nb,
+                            _stream_handle(stream))
+        return Y
+
+    def export(self):
+        """Host copies of the prepared weight in logical layouts (numpy arrays)."""
+        import numpy as np
+        codes = np.empty((self.N, self.K // 2), np.uint8)
+        scales = np.empty((self.N, self.K // 16), np.uint8)
+        L1 = np.empty((self.K, self.r), np.uint16)
+        L2t = np.empty((self.N, self.r), np.uint16)
+        inv = np.empty(self.K, np.float32)
+        svdq_weight_export(self.w, codes.ctypes.data, scales.ctypes.data,
+                           L1.ctypes.data if self.r else 0, L2t.ctypes.data if self.r else 0,
+                           inv.ctypes.data, _stream_handle())
+        return dict(w_codes=codes, w_scales=scales, L1=L1, L2t=L2t, inv_lambda=inv)

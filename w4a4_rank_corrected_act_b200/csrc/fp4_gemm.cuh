@@ -1,0 +1,309 @@
+// fp4_gemm.cuh -- block-scaled NVFP4 GEMM with the low-rank branch fused,
+// on the 5th-generation tensor cores (tcgen05) of sm_100a.
+//
+//   Y = bf16( D . L2  +  deq(Xq) . deq(Rq)^T  +  bias )
+//
+// "Most operations happen in 4-bit tensor cores, while the low-rank correction
+// runs in higher precision" (imaginepro.ai "Nunchaku 4-Bit Diffusion Inference
+// in Diffusers: A Practical Guide", section "Under the Hood"); NVFP4 is the
+// Blackwell/B200 precision (chaosnode.de "Nunchaku Lite", section
+// "Hardware-Support").
+//
+// Per 128 x BN output tile, one fp32 accumulator lives in tensor memory:
+//   1. the low-rank term: R_PAD/16 bf16 MMAs (kind::f16, K = 16) of the D tile
+//      (128 x r) against the L2^T tile (BN x r) initialise the accumulator;
+//   2. K/64 block-scaled MMAs (kind::mxf4nvf4, K = 64, one UE4M3 scale per 16)
+//      accumulate the 4-bit product; scales are copied shared -> tensor memory
+//      with tcgen05.cp right before the MMAs that read them;
+//   3. the epilogue reads the accumulator with tcgen05.ld, adds the bias,
+//      rounds to bf16 and stores Y.
+// Warp roles (256 threads): warp 0 issues TMA / bulk copies into a STAGES-deep
+// shared-memory ring, warp 1 issues the MMAs (one thread), warp 2 owns the
+// tensor-memory allocation, warps 4-7 run the epilogue (warp w reads lanes
+// 32*(w%4)..+31).  The grid is persistent (one CTA per SM, tiles strided).
+#pragma once
+
+#include "nvfp4.cuh"
+#include "ptx.cuh"
+
+namespace svdq {
+
+constexpr int GEMM_BM = 128;
+constexpr int GEMM_BK = 256;                 // fp4 elements per stage = 128 bytes per row
+constexpr int GEMM_THREADS = 256;
+constexpr uint32_t GEMM_A_TILE = GEMM_BM * 128;   // 16 KB
+constexpr uint32_t GEMM_SFA_TILE = 4 * 512;       // 4 scale tiles (4 x 64 K) for 128 rows
+
+struct GemmParams {
+  const uint8_t* x_scales;
+  const uint8_t* w_scales;
+  const uint16_t* bias;
+  uint16_t* Y;
+  int M, N, K, r;
+  int m_tiles, n_tiles, num_tiles, kblocks;
+};
+
+template <int BN>
+struct GemmCfg {
+  static constexpr uint32_t kBTile = BN * 128;
+  static constexpr uint32_t kSFBTile = (BN / 128) * GEMM_SFA_TILE;
+  static constexpr uint32_t kStage = GEMM_A_TILE + kBTile + GEMM_SFA_TILE + kSFBTile;
+  static constexpr int kStages = (BN == 256 ? 4 : 6);
+  static constexpr uint32_t kSfColsPerStage = 16 + BN / 8;   // SFA 4x4 + SFB 4x(BN/32)
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kBarBytes = (2 * kStages + 3) * 8 + 16;
+  static constexpr uint32_t kSmemBytes = kStages * kStage + kBarBytes + 1024;
+  static_assert(BN + kStages * kSfColsPerStage <= kTmemCols, "tensor memory budget");
+  static_assert(kStage % 1024 == 0, "stage alignment");
+};
+
+// Instruction descriptors (tcgen05.mma, 32-bit):
+//   kind::f16      : bits 4-5 D format (1 = f32), 7-9 A format (1 = bf16),
+//                    10-12 B format (1 = bf16), 15/16 A/B major (0 = K-major),
+//                    17-22 N >> 3, 24-28 M >> 4.
+//   kind::mxf4nvf4 : bits 4-5 B scale id, 7-9 A format (1 = E2M1), 10-12 B
+//                    format (1 = E2M1), 17-22 N >> 3, 23 scale type (0 = UE4M3),
+//                    24-28 M >> 4, 29-30 A scale id, 31 K size (0 = 64).
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+__host__ __device__ constexpr uint32_t idesc_nvfp4(int M, int N) {
+  return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+template <int BN, int R_PAD>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    fp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                    const __grid_constant__ CUtensorMap tm_d, const __grid_constant__ CUtensorMap tm_l2,
+                    const GemmParams p) {
+  using Cfg = GemmCfg<BN>;
+  constexpr int S = Cfg::kStages;
+  constexpr uint32_t kLRLayout = (R_PAD == 64 ? LAYOUT_SW128 : R_PAD == 32 ? LAYOUT_SW64 : LAYOUT_SW32);
+  constexpr uint32_t kLRSbo = 8 * R_PAD * 2;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * Cfg::kStage);
+  // bars[0..S): full, [S..2S): empty, 2S: tmem_full, 2S+1: tmem_empty, 2S+2: drain
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 3);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t smem_base = smem_u32(smem);
+  auto stage_a = [&](int s) { return smem_base + s * Cfg::kStage; };
+  auto stage_b = [&](int s) { return smem_base + s * Cfg::kStage + GEMM_A_TILE; };
+  auto stage_sfa = [&](int s) { return smem_base + s * Cfg::kStage + GEMM_A_TILE + Cfg::kBTile; };
+  auto stage_sfb = [&](int s) {
+    return smem_base + s * Cfg::kStage + GEMM_A_TILE + Cfg::kBTile + GEMM_SFA_TILE;
+  };
+  auto full_bar = [&](int s) { return smem_u32(bars + s); };
+  auto empty_bar = [&](int s) { return smem_u32(bars + S + s); };
+  const uint32_t tmem_full = smem_u32(bars + 2 * S);
+  const uint32_t tmem_empty = smem_u32(bars + 2 * S + 1);
+  const uint32_t drain_bar = smem_u32(bars + 2 * S + 2);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    mbar_init(tmem_full, 1);
+    mbar_init(tmem_empty, 128);
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(smem_u32(tmem_slot), Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int kb_per_tile = p.kblocks;
+  const uint32_t k_tiles64 = static_cast<uint32_t>(p.K) >> 6;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_a);
+      tma_prefetch_desc(&tm_b);
+      if (R_PAD > 0) {
+        tma_prefetch_desc(&tm_d);
+        tma_prefetch_desc(&tm_l2);
+      }
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      int8_t fill_parity[S];
+      for (int s = 0; s < S; ++s) fill_parity[s] = -1;
+      const uint32_t tx_main = GEMM_A_TILE + Cfg::kBTile + GEMM_SFA_TILE + Cfg::kSFBTile;
+      const uint32_t tx_lr = (GEMM_BM + BN) * R_PAD * 2;
+      bool ok = true;
+      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+        const int mb = t % p.m_tiles, nb = t / p.m_tiles;
+        const int m0 = mb * GEMM_BM, n0 = nb * BN;
+        if (R_PAD > 0) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1, abort_flag, KID_GEMM, 1)) { ok = false; break; }
+          mbar_arrive_expect_tx(full_bar(stage), tx_lr);
+          tma_load_2d(stage_a(stage), &tm_d, full_bar(stage), 0, m0);
+          tma_load_2d(stage_b(stage), &tm_l2, full_bar(stage), 0, n0);
+          fill_parity[stage] = static_cast<int8_t>(phase);
+          ++issued;
+          if (++stage == S) { stage = 0; phase ^= 1; }
+        }
+        for (int kb = 0; kb < kb_per_tile; ++kb) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1, abort_flag, KID_GEMM, 2)) { ok = false; break; }
+          mbar_arrive_expect_tx(full_bar(stage), tx_main);
+          tma_load_2d(stage_a(stage), &tm_a, full_bar(stage), kb * 128, m0);
+          tma_load_2d(stage_b(stage), &tm_b, full_bar(stage), kb * 128, n0);
+          bulk_load(stage_sfa(stage),
+                    p.x_scales + (static_cast<size_t>(mb) * k_tiles64 + kb * 4) * 512,
+                    GEMM_SFA_TILE, full_bar(stage));
+#pragma unroll
+          for (int g = 0; g < BN / 128; ++g)
+            bulk_load(stage_sfb(stage) + g * GEMM_SFA_TILE,
+                      p.w_scales + (static_cast<size_t>(n0 / 128 + g) * k_tiles64 + kb * 4) * 512,
+                      GEMM_SFA_TILE, full_bar(stage));
+          fill_parity[stage] = static_cast<int8_t>(phase);
+          ++issued;
+          if (++stage == S) { stage = 0; phase ^= 1; }
+        }
+      }
+      if (*abort_flag) {
+        for (int s = 0; s < S; ++s)
+          if (fill_parity[s] >= 0)
+            mbar_wait_drain(full_bar(s), static_cast<uint32_t>(fill_parity[s]));
+      }
+      (void)issued;
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idf = idesc_nvfp4(GEMM_BM, BN);
+      const uint32_t idb = idesc_bf16(GEMM_BM, BN);
+      int stage = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      bool any_issued = false;
+      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+        if (!mbar_wait(tmem_empty, acc_phase ^ 1, abort_flag, KID_GEMM, 4)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t accumulate = 0;
+        if (R_PAD > 0) {
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, KID_GEMM, 5)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t ad = make_smem_desc(stage_a(stage), kLRLayout, kLRSbo, 0);
+          const uint64_t bd = make_smem_desc(stage_b(stage), kLRLayout, kLRSbo, 0);
+#pragma unroll
+          for (int kk = 0; kk < R_PAD / 16; ++kk) {
+            tc_mma_bf16(tmem_base, ad + 2 * kk, bd + 2 * kk, idb, accumulate);
+            accumulate = 1;
+          }
+          tc_commit(empty_bar(stage));
+          any_issued = true;
+          if (++stage == S) { stage = 0; phase ^= 1; }
+        }
+        for (int kb = 0; kb < kb_per_tile; ++kb) {
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, KID_GEMM, 6)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sf_cols = BN + stage * Cfg::kSfColsPerStage;
+          // scale factors: shared -> tensor memory (32 rows x 16 B per copy)
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            tc_cp_32x128b_warpx4(tmem_base + sf_cols + 4 * i,
+                                 make_smem_desc(stage_sfa(stage) + i * 512, LAYOUT_NONE, 128, 0));
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int g = 0; g < BN / 128; ++g)
+              tc_cp_32x128b_warpx4(
+                  tmem_base + sf_cols + 16 + i * (BN / 32) + 4 * g,
+                  make_smem_desc(stage_sfb(stage) + (g * 4 + i) * 512, LAYOUT_NONE, 128, 0));
+          const uint64_t ad = make_smem_desc(stage_a(stage), LAYOUT_SW128, 1024, 0);
+          const uint64_t bd = make_smem_desc(stage_b(stage), LAYOUT_SW128, 1024, 0);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            tc_mma_nvfp4(tmem_base, ad + 2 * i, bd + 2 * i, idf, tmem_base + sf_cols + 4 * i,
+                         tmem_base + sf_cols + 16 + i * (BN / 32), accumulate);
+            accumulate = 1;
+          }
+          tc_commit(empty_bar(stage));
+          any_issued = true;
+          if (++stage == S) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        tc_commit(tmem_full);
+        acc_phase ^= 1;
+      }
+      if (*abort_flag && any_issued) {
+        // make sure no MMA still writes tensor memory before it is freed
+        tc_commit(drain_bar);
+        mbar_wait_drain(drain_bar, 0);
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
+      const int mb = t % p.m_tiles, nb = t / p.m_tiles;
+      const int m0 = mb * GEMM_BM, n0 = nb * BN;
+      if (!mbar_wait(tmem_full, acc_phase, abort_flag, KID_GEMM, 8)) break;
+      tc_fence_after();
+      const int row = m0 + q * 32 + lane;
+      uint16_t* yrow = p.Y + static_cast<size_t>(row) * p.N + n0;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + c * 32, v);
+        tmem_ld_wait();
+        float f[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[j]);
+        if (p.bias != nullptr) {
+          const uint4* bp = reinterpret_cast<const uint4*>(p.bias + n0 + c * 32);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const uint4 b = __ldg(bp + u);
+            const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              f[u * 8 + 2 * h] += bf16_bits_to_f32(bw[h] & 0xFFFFu);
+              f[u * 8 + 2 * h + 1] += bf16_bits_to_f32(bw[h] >> 16);
+            }
+          }
+        }
+        if (row < p.M) {
+          uint4* dst = reinterpret_cast<uint4*>(yrow + c * 32);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            uint4 o;
+            o.x = pack_bf16x2(f[u * 8 + 0], f[u * 8 + 1]);
+            o.y = pack_bf16x2(f[u * 8 + 2], f[u * 8 + 3]);
+            o.z = pack_bf16x2(f[u * 8 + 4], f[u * 8 + 5]);
+            o.w = pack_bf16x2(f[u * 8 + 6], f[u * 8 + 7]);
+            dst[u] = o;
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(tmem_empty);
+      acc_phase ^= 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cfg::kTmemCols);
+  }
+}
+
+}  // namespace svdq

@@ -1,0 +1,107 @@
+// nvfp4.cuh -- NVFP4 block quantiser (device side).
+//
+// Format (the 4-bit precision listed for Blackwell / B200 in chaosnode.de
+// "Nunchaku Lite: 4-Bit Diffusion-Inferenz direkt in Diffusers", section
+// "Hardware-Support"): E2M1 element codes {0,.5,1,1.5,2,3,4,6} x sign, one
+// E4M3 scale per 16 consecutive elements along K.  For a block v[0..15]:
+//     a = max|v_i|,  s = E4M3_rn_satfinite(f32(a / 6)),
+//     q_i = E2M1_rn_satfinite(f32(v_i / s))   (q_i = +-0 when s == 0),
+// with IEEE float32 division, round-to-nearest-even conversions, and the sign
+// bit of E2M1 kept (a negative value that rounds to zero is code 0x8).
+// Codes are packed two per byte, element 2j in the low nibble of byte j.
+#pragma once
+
+#include <stdint.h>
+
+namespace svdq {
+
+// E4M3 code (0x00..0x7E) of a non-negative float, RNE, saturating at 448.
+__device__ __forceinline__ uint32_t e4m3_rn_satfinite(float x) {
+  uint16_t out;
+  asm("{\n\t.reg .b16 t;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 t, %1, %2;\n\t"
+      "mov.b16 %0, t;\n\t}\n"
+      : "=h"(out)
+      : "f"(0.0f), "f"(x));
+  return static_cast<uint32_t>(out) & 0xFFu;
+}
+
+// Exact float value of a non-negative E4M3 code.
+__device__ __forceinline__ float e4m3_to_f32(uint32_t c) {
+  const uint32_t e = (c >> 3) & 15u, m = c & 7u;
+  if (e == 0) return static_cast<float>(m) * 0x1p-9f;
+  return __uint_as_float(((e + 120u) << 23) | (m << 20));
+}
+
+// Eight E2M1 magnitude codes of |q0..q7| (RNE, satfinite), packed with q0 in
+// the lowest nibble; sign bits are added by the caller.
+__device__ __forceinline__ uint32_t e2m1x8_magnitudes(const float (&a)[8]) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}\n"
+      : "=r"(out)
+      : "f"(a[0]), "f"(a[1]), "f"(a[2]), "f"(a[3]), "f"(a[4]), "f"(a[5]), "f"(a[6]),
+        "f"(a[7]));
+  return out;
+}
+
+// Quantise 8 consecutive values forming one half of a 16-element block; the
+// other half lives on lane (laneid ^ 1).  Must be called by all 32 lanes of
+// the warp.  Returns the 8 packed codes; `scale_code` receives the block's
+// E4M3 code (identical on both lanes of the pair).
+__device__ __forceinline__ uint32_t nvfp4_quant_half_block(const float (&v)[8],
+                                                          uint32_t& scale_code) {
+  float am = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(v[i]));
+  am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+  const uint32_t sc = e4m3_rn_satfinite(__fdiv_rn(am, 6.0f));
+  const float s = e4m3_to_f32(sc);
+  float mag[8];
+  uint32_t signs = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float q = (s == 0.0f) ? 0.0f : __fdiv_rn(v[i], s);
+    mag[i] = fabsf(q);
+    signs |= (__float_as_uint(v[i]) >> 31) << (4 * i + 3);
+  }
+  scale_code = sc;
+  return e2m1x8_magnitudes(mag) | signs;
+}
+
+// Byte offset of scale (row, kb16) in the scale-factor tile layout:
+// 512-byte tiles of 128 rows x 4 scales, tile (row/128, kb16/4) at
+// ((row/128) * (K/64) + kb16/4) * 512, inside it (row%32)*16 + ((row/32)%4)*4 + kb16%4.
+__host__ __device__ __forceinline__ uint64_t sf_offset(uint32_t row, uint32_t kb16, uint32_t K) {
+  const uint64_t tile = static_cast<uint64_t>(row >> 7) * (K >> 6) + (kb16 >> 2);
+  return tile * 512u + (row & 31u) * 16u + ((row >> 5) & 3u) * 4u + (kb16 & 3u);
+}
+
+// Round float64 to bf16 (RNE, single rounding); returns the bit pattern.
+__device__ __forceinline__ uint16_t f64_to_bf16_rne(double x) {
+  if (fabs(x) < 0x1p-126) {
+    // bf16 subnormal range: multiples of 2^-133, ties to even (rint).
+    const float f = static_cast<float>(rint(x * 0x1p133) * 0x1p-133);
+    return static_cast<uint16_t>(__float_as_uint(f) >> 16);
+  }
+  unsigned long long u = static_cast<unsigned long long>(__double_as_longlong(x));
+  const unsigned long long lsb = (u >> 45) & 1ull;
+  u = (u + ((1ull << 44) - 1ull) + lsb) & ~((1ull << 45) - 1ull);
+  const float f = static_cast<float>(__longlong_as_double(static_cast<long long>(u)));
+  return static_cast<uint16_t>(__float_as_uint(f) >> 16);
+}
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as_float(b << 16); }
+
+// Two floats -> packed bf16x2 (RNE), first argument in the low half.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t out;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(out) : "f"(hi), "f"(lo));
+  return out;
+}
+
+}  // namespace svdq

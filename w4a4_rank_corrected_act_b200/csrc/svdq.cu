@@ -1,0 +1,647 @@
+// svdq.cu -- C ABI of the B200 SVDQuant W4A4 linear layer (host side) and the
+// single translation unit that holds every device kernel of the library.
+//
+// The entry points mirror the statement of the problem on the pages: a
+// drop-in replacement of a linear layer whose weights are quantised offline
+// (chaosnode.de "Nunchaku Lite: 4-Bit Diffusion-Inferenz direkt in
+// Diffusers", section "Nunchaku Lite vs. Original": runtime SVDQ layers in
+// place of nn.Linear; watch-ia.com: quantise, package, load and verify) and
+// run W4A4 at inference (aiphreaks.com "Bringing Nunchaku 4-bit Diffusion
+// Inference to Diffusers", section "Technical Breakdown and Performance
+// Metrics").  Argument meaning, layouts and error behaviour: include/svdq.h.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+#include <cusolverDn.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "svdq.h"
+#include "act_quant.cuh"
+#include "fp4_gemm.cuh"
+#include "prepare.cuh"
+
+using namespace svdq;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+svdq_status cuda_fail(cudaError_t e, const char* what) {
+  g_last_error = std::string(what) + ": " + cudaGetErrorName(e) + " (" + cudaGetErrorString(e) + ")";
+  return SVDQ_ERR_CUDA;
+}
+
+#define SVDQ_CUDA(call)                                   \
+  do {                                                    \
+    cudaError_t e_ = (call);                              \
+    if (e_ != cudaSuccess) return cuda_fail(e_, #call);   \
+  } while (0)
+
+#define SVDQ_CHECK_LAUNCH(name)                           \
+  do {                                                    \
+    cudaError_t e_ = cudaGetLastError();                  \
+    if (e_ != cudaSuccess) return cuda_fail(e_, name);    \
+  } while (0)
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int r_pad_of(int r) { return r == 0 ? 0 : r <= 16 ? 16 : r <= 32 ? 32 : 64; }
+
+// Shape check shared by every entry point (see the header for the rules).
+svdq_status check_layer_shape(int N, int K, int r) {
+  if (N <= 0 || K <= 0 || r < 0 || (K % 16) != 0) return SVDQ_ERR_INVALID_ARG;
+  if ((K % 256) != 0 || (N % 128) != 0 || (r % 8) != 0 || r > 64 || r > std::min(N, K))
+    return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  return SVDQ_OK;
+}
+
+svdq_status check_weight(const svdq_weight* w) {
+  if (w == nullptr) return SVDQ_ERR_INVALID_ARG;
+  svdq_status s = check_layer_shape(w->N, w->K, w->r);
+  if (s != SVDQ_OK) return s;
+  if (w->w_codes == nullptr || w->w_scales == nullptr || w->inv_lambda == nullptr)
+    return SVDQ_ERR_INVALID_ARG;
+  if (w->r > 0 && (w->L1 == nullptr || w->L2t == nullptr)) return SVDQ_ERR_INVALID_ARG;
+  if (w->has_bias && w->bias == nullptr) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(w->w_codes) || !aligned16(w->w_scales) || !aligned16(w->inv_lambda) ||
+      (w->r > 0 && (!aligned16(w->L1) || !aligned16(w->L2t))) ||
+      (w->has_bias && !aligned16(w->bias)))
+    return SVDQ_ERR_MISALIGNED;
+  return SVDQ_OK;
+}
+
+int m_pad_of(int M) { return (M + 127) / 128 * 128; }
+
+// --------------------------------------------------------------------------
+// TMA descriptor encoding through the driver entry point (no libcuda link).
+// --------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D row-major tensor: `inner` elements per row (contiguous), `rows` rows,
+// row pitch `pitch_bytes`; box `box_inner` x `box_rows`.
+svdq_status make_tmap(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner,
+                      uint64_t rows, uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_rows,
+                      CUtensorMapSwizzle swz) {
+  auto fn = encode_fn();
+  if (fn == nullptr) {
+    g_last_error = "cuTensorMapEncodeTiled entry point unavailable";
+    return SVDQ_ERR_CUDA;
+  }
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {pitch_bytes};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    char buf[160];
+    std::snprintf(buf, sizeof(buf), "cuTensorMapEncodeTiled failed (%d) inner=%llu rows=%llu box=%ux%u",
+                  static_cast<int>(r), static_cast<unsigned long long>(inner),
+                  static_cast<unsigned long long>(rows), box_inner, box_rows);
+    g_last_error = buf;
+    return SVDQ_ERR_CUDA;
+  }
+  return SVDQ_OK;
+}
+
+CUtensorMapSwizzle lr_swizzle(int r_pad) {
+  return r_pad == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
+                     : r_pad == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+}
+
+int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+// --------------------------------------------------------------------------
+// Launchers
+// --------------------------------------------------------------------------
+template <int R_PAD>
+svdq_status launch_act(const CUtensorMap& tx, const CUtensorMap& tl1, const ActParams& p,
+                       cudaStream_t st) {
+  const uint32_t smem = ActSmem<R_PAD>::bytes(p.stages);
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(act_quant_kernel<R_PAD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    227 * 1024);
+  });
+  if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(act)");
+  const int grid = p.M_pad / ACT_BM;
+  act_quant_kernel<R_PAD><<<grid, ACT_THREADS, smem, st>>>(tx, tl1, p);
+  SVDQ_CHECK_LAUNCH("act_quant_kernel");
+  return SVDQ_OK;
+}
+
+template <int BN, int R_PAD>
+svdq_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
+                        const CUtensorMap& tl2, const GemmParams& p, cudaStream_t st) {
+  using Cfg = GemmCfg<BN>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(fp4_gemm_kernel<BN, R_PAD>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
+  });
+  if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(gemm)");
+  const int grid = std::min(p.num_tiles, num_sms());
+  fp4_gemm_kernel<BN, R_PAD><<<grid, GEMM_THREADS, Cfg::kSmemBytes, st>>>(ta, tb, td, tl2, p);
+  SVDQ_CHECK_LAUNCH("fp4_gemm_kernel");
+  return SVDQ_OK;
+}
+
+template <int BN>
+svdq_status dispatch_gemm_r(int r_pad, const CUtensorMap& ta, const CUtensorMap& tb,
+                            const CUtensorMap& td, const CUtensorMap& tl2, const GemmParams& p,
+                            cudaStream_t st) {
+  switch (r_pad) {
+    case 0: return launch_gemm<BN, 0>(ta, tb, td, tl2, p, st);
+    case 16: return launch_gemm<BN, 16>(ta, tb, td, tl2, p, st);
+    case 32: return launch_gemm<BN, 32>(ta, tb, td, tl2, p, st);
+    default: return launch_gemm<BN, 64>(ta, tb, td, tl2, p, st);
+  }
+}
+
+int act_stages(int r_pad) {
+  // as many 16 KB + L1-slice stages as fit next to the reduction buffer (max 4)
+  const uint32_t budget = 227 * 1024;
+  for (int s = 4; s >= 2; --s) {
+    uint32_t b = 0;
+    switch (r_pad) {
+      case 0: b = ActSmem<0>::bytes(s); break;
+      case 16: b = ActSmem<16>::bytes(s); break;
+      case 32: b = ActSmem<32>::bytes(s); break;
+      default: b = ActSmem<64>::bytes(s); break;
+    }
+    if (b <= budget) return s;
+  }
+  return 2;
+}
+
+svdq_status quantize_act_impl(const uint16_t* X, int M, const svdq_weight* w, uint8_t* x_codes,
+                              uint8_t* x_scales, uint16_t* D, cudaStream_t st) {
+  const int K = w->K, r = w->r, rp = r_pad_of(r);
+  CUtensorMap tx{}, tl1{};
+  svdq_status s = make_tmap(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M,
+                            static_cast<uint64_t>(K) * 2, 64, ACT_BM, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (s != SVDQ_OK) return s;
+  if (r > 0) {
+    s = make_tmap(&tl1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->L1, r, K, static_cast<uint64_t>(r) * 2,
+                  rp, ACT_KC, lr_swizzle(rp));
+    if (s != SVDQ_OK) return s;
+  }
+  ActParams p;
+  p.inv_lambda = w->inv_lambda;
+  p.x_codes = x_codes;
+  p.x_scales = x_scales;
+  p.D = D;
+  p.M = M;
+  p.K = K;
+  p.r = r;
+  p.M_pad = m_pad_of(M);
+  p.stages = act_stages(rp);
+  switch (rp) {
+    case 0: return launch_act<0>(tx, tl1, p, st);
+    case 16: return launch_act<16>(tx, tl1, p, st);
+    case 32: return launch_act<32>(tx, tl1, p, st);
+    default: return launch_act<64>(tx, tl1, p, st);
+  }
+}
+
+svdq_status gemm_impl(const uint8_t* x_codes, const uint8_t* x_scales, const uint16_t* D, int M,
+                      const svdq_weight* w, uint16_t* Y, cudaStream_t st) {
+  const int N = w->N, K = w->K, r = w->r, rp = r_pad_of(r);
+  const int m_tiles = (M + GEMM_BM - 1) / GEMM_BM;
+  // 256-wide tiles when N allows it and there are enough of them to fill the GPU
+  int BN = (N % 256 == 0) ? 256 : 128;
+  if (BN == 256 && m_tiles * (N / 256) < num_sms()) BN = 128;
+  if (const char* e = std::getenv("SVDQ_GEMM_BN")) {   // tile-width override (128 or 256)
+    const int v = std::atoi(e);
+    if (v == 128 || (v == 256 && N % 256 == 0)) BN = v;
+  }
+  CUtensorMap ta{}, tb{}, td{}, tl2{};
+  svdq_status s = make_tmap(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, x_codes, K / 2, M, K / 2, 128,
+                            GEMM_BM, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (s != SVDQ_OK) return s;
+  s = make_tmap(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->w_codes, K / 2, N, K / 2, 128, BN,
+                CU_TENSOR_MAP_SWIZZLE_128B);
+  if (s != SVDQ_OK) return s;
+  if (r > 0) {
+    s = make_tmap(&td, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, D, r, M, static_cast<uint64_t>(r) * 2, rp,
+                  GEMM_BM, lr_swizzle(rp));
+    if (s != SVDQ_OK) return s;
+    s = make_tmap(&tl2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->L2t, r, N,
+                  static_cast<uint64_t>(r) * 2, rp, BN, lr_swizzle(rp));
+    if (s != SVDQ_OK) return s;
+  }
+  GemmParams p;
+  p.x_scales = x_scales;
+  p.w_scales = w->w_scales;
+  p.bias = w->has_bias ? w->bias : nullptr;
+  p.Y = Y;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.r = r;
+  p.m_tiles = m_tiles;
+  p.n_tiles = N / BN;
+  p.num_tiles = p.m_tiles * p.n_tiles;
+  p.kblocks = K / GEMM_BK;
+  return BN == 256 ? dispatch_gemm_r<256>(rp, ta, tb, td, tl2, p, st)
+                   : dispatch_gemm_r<128>(rp, ta, tb, td, tl2, p, st);
+}
+
+struct ActWs {
+  uint8_t* codes;
+  uint8_t* scales;
+  uint16_t* D;
+};
+
+size_t act_ws_layout(int M, int K, int r, uint8_t* base, ActWs* out) {
+  const size_t c = align_up(static_cast<size_t>(M) * (K / 2), kAlign);
+  const size_t s = align_up(static_cast<size_t>(m_pad_of(M)) * (K / 16), kAlign);
+  const size_t d = align_up(static_cast<size_t>(M) * r * 2, kAlign);
+  if (out != nullptr) {
+    out->codes = base;
+    out->scales = base + c;
+    out->D = r > 0 ? reinterpret_cast<uint16_t*>(base + c + s) : nullptr;
+  }
+  return c + s + d;
+}
+
+// Weight buffer layout, each field 256-byte aligned.
+size_t weight_layout(int N, int K, int r, int has_bias, uint8_t* base, svdq_weight* out) {
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align_up(bytes, kAlign);
+    return base == nullptr ? nullptr : base + o;
+  };
+  uint8_t* codes = take(static_cast<size_t>(N) * (K / 2));
+  uint8_t* scales = take(static_cast<size_t>(N) * (K / 16));
+  uint8_t* l1 = take(static_cast<size_t>(K) * r * 2);
+  uint8_t* l2t = take(static_cast<size_t>(N) * r * 2);
+  uint8_t* inv = take(static_cast<size_t>(K) * 4);
+  uint8_t* bias = has_bias ? take(static_cast<size_t>(N) * 2) : nullptr;
+  if (out != nullptr) {
+    out->N = N;
+    out->K = K;
+    out->r = r;
+    out->has_bias = has_bias ? 1 : 0;
+    out->w_codes = codes;
+    out->w_scales = scales;
+    out->L1 = r > 0 ? reinterpret_cast<uint16_t*>(l1) : nullptr;
+    out->L2t = r > 0 ? reinterpret_cast<uint16_t*>(l2t) : nullptr;
+    out->inv_lambda = reinterpret_cast<float*>(inv);
+    out->bias = reinterpret_cast<uint16_t*>(bias);
+  }
+  return off;
+}
+
+struct PrepWs {
+  float* what;
+  double* G;
+  double* ev;
+  double* L1f;
+  double* L2f;
+  double* work;
+  int* info;
+  int lwork;
+};
+
+size_t prep_ws_layout(int N, int K, int r, int lwork, uint8_t* base, PrepWs* out) {
+  const int n = std::min(N, K);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align_up(bytes, kAlign);
+    return base == nullptr ? nullptr : base + o;
+  };
+  uint8_t* what = take(static_cast<size_t>(N) * K * 4);
+  uint8_t* G = take(r > 0 ? static_cast<size_t>(n) * n * 8 : 0);
+  uint8_t* ev = take(r > 0 ? static_cast<size_t>(n) * 8 : 0);
+  uint8_t* l1 = take(static_cast<size_t>(K) * r * 8);
+  uint8_t* l2 = take(static_cast<size_t>(N) * r * 8);
+  uint8_t* work = take(r > 0 ? static_cast<size_t>(lwork) * 8 : 0);
+  uint8_t* info = take(16);
+  if (out != nullptr) {
+    out->what = reinterpret_cast<float*>(what);
+    out->G = reinterpret_cast<double*>(G);
+    out->ev = reinterpret_cast<double*>(ev);
+    out->L1f = reinterpret_cast<double*>(l1);
+    out->L2f = reinterpret_cast<double*>(l2);
+    out->work = reinterpret_cast<double*>(work);
+    out->info = reinterpret_cast<int*>(info);
+    out->lwork = lwork;
+  }
+  return off;
+}
+
+int syevd_lwork(int n, cusolverDnHandle_t h) {
+  int lwork = 0;
+  if (cusolverDnDsyevd_bufferSize(h, CUSOLVER_EIG_MODE_VECTOR, CUBLAS_FILL_MODE_LOWER, n, nullptr, n,
+                                  nullptr, &lwork) != CUSOLVER_STATUS_SUCCESS)
+    return -1;
+  return lwork;
+}
+
+void to_logical(const uint8_t* native, int rows, int K, uint8_t* logical) {
+  const int kb = K / 16;
+  for (int i = 0; i < rows; ++i)
+    for (int j = 0; j < kb; ++j)
+      logical[static_cast<size_t>(i) * kb + j] = native[sf_offset(i, j, K)];
+}
+
+}  // namespace
+
+// ==========================================================================
+// C ABI
+// ==========================================================================
+extern "C" {
+
+const char* svdq_status_string(svdq_status s) {
+  switch (s) {
+    case SVDQ_OK: return "SVDQ_OK";
+    case SVDQ_ERR_INVALID_ARG: return "SVDQ_ERR_INVALID_ARG";
+    case SVDQ_ERR_UNSUPPORTED_SHAPE: return "SVDQ_ERR_UNSUPPORTED_SHAPE";
+    case SVDQ_ERR_MISALIGNED: return "SVDQ_ERR_MISALIGNED";
+    case SVDQ_ERR_WORKSPACE_TOO_SMALL: return "SVDQ_ERR_WORKSPACE_TOO_SMALL";
+    case SVDQ_ERR_CUDA: return "SVDQ_ERR_CUDA";
+    case SVDQ_ERR_TIMEOUT: return "SVDQ_ERR_TIMEOUT";
+    case SVDQ_ERR_SOLVER: return "SVDQ_ERR_SOLVER";
+  }
+  return "SVDQ_ERR_UNKNOWN";
+}
+
+const char* svdq_last_error_detail(void) { return g_last_error.c_str(); }
+
+const char* svdq_version(void) { return "svdq-b200 0.1 (sm_100a)"; }
+
+size_t svdq_weight_bytes(int N, int K, int r, int has_bias) {
+  if (check_layer_shape(N, K, r) != SVDQ_OK) return 0;
+  return weight_layout(N, K, r, has_bias, nullptr, nullptr);
+}
+
+size_t svdq_act_codes_bytes(int M, int K) {
+  if (M < 0 || K <= 0 || K % 16) return 0;
+  return static_cast<size_t>(M) * (K / 2);
+}
+
+size_t svdq_act_scales_bytes(int M, int K) {
+  if (M < 0 || K <= 0 || K % 64) return 0;
+  return static_cast<size_t>(m_pad_of(M)) * (K / 16);
+}
+
+size_t svdq_forward_workspace_bytes(int M, int N, int K, int r) {
+  if (M < 0 || check_layer_shape(N, K, r) != SVDQ_OK) return 0;
+  return act_ws_layout(M, K, r, nullptr, nullptr);
+}
+
+size_t svdq_prepare_workspace_bytes(int N, int K, int r) {
+  if (check_layer_shape(N, K, r) != SVDQ_OK) return 0;
+  int lwork = 0;
+  if (r > 0) {
+    cusolverDnHandle_t h = nullptr;
+    if (cusolverDnCreate(&h) != CUSOLVER_STATUS_SUCCESS) return 0;
+    lwork = syevd_lwork(std::min(N, K), h);
+    cusolverDnDestroy(h);
+    if (lwork < 0) return 0;
+  }
+  return prep_ws_layout(N, K, r, lwork, nullptr, nullptr);
+}
+
+svdq_status svdq_weight_bind(void* buf, size_t bytes, int N, int K, int r, int has_bias,
+                             svdq_weight* out) {
+  if (buf == nullptr || out == nullptr) return SVDQ_ERR_INVALID_ARG;
+  svdq_status s = check_layer_shape(N, K, r);
+  if (s != SVDQ_OK) return s;
+  if ((reinterpret_cast<uintptr_t>(buf) & (kAlign - 1)) != 0) return SVDQ_ERR_MISALIGNED;
+  if (bytes < weight_layout(N, K, r, has_bias, nullptr, nullptr)) return SVDQ_ERR_WORKSPACE_TOO_SMALL;
+  weight_layout(N, K, r, has_bias, static_cast<uint8_t*>(buf), out);
+  return SVDQ_OK;
+}
+
+svdq_status svdq_prepare_weight(const uint16_t* W, const float* lambda, const uint16_t* bias,
+                                const svdq_weight* w, void* ws, size_t ws_bytes, void* stream) {
+  svdq_status s = check_weight(w);
+  if (s != SVDQ_OK) return s;
+  if (W == nullptr || lambda == nullptr || ws == nullptr) return SVDQ_ERR_INVALID_ARG;
+  if ((bias != nullptr) != (w->has_bias != 0)) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(lambda) || (bias && !aligned16(bias)) || !aligned16(ws))
+    return SVDQ_ERR_MISALIGNED;
+  const int N = w->N, K = w->K, r = w->r, n = std::min(N, K);
+  const int col_gram = K <= N ? 1 : 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  cusolverDnHandle_t h = nullptr;
+  int lwork = 0;
+  if (r > 0) {
+    if (cusolverDnCreate(&h) != CUSOLVER_STATUS_SUCCESS) {
+      g_last_error = "cusolverDnCreate failed";
+      return SVDQ_ERR_SOLVER;
+    }
+    lwork = syevd_lwork(n, h);
+    if (lwork < 0) {
+      cusolverDnDestroy(h);
+      g_last_error = "cusolverDnDsyevd_bufferSize failed";
+      return SVDQ_ERR_SOLVER;
+    }
+  }
+  PrepWs pw;
+  if (ws_bytes < prep_ws_layout(N, K, r, lwork, nullptr, nullptr)) {
+    if (h) cusolverDnDestroy(h);
+    return SVDQ_ERR_WORKSPACE_TOO_SMALL;
+  }
+  prep_ws_layout(N, K, r, lwork, static_cast<uint8_t*>(ws), &pw);
+
+  auto fail = [&](svdq_status e) {
+    if (h) cusolverDnDestroy(h);
+    return e;
+  };
+
+  const int nsm = num_sms();
+  prep_smooth_kernel<<<nsm * 8, 256, 0, st>>>(W, lambda, bias, N, K, pw.what, w->inv_lambda,
+                                              w->has_bias ? w->bias : nullptr);
+  {
+    cudaError_t e0 = cudaGetLastError();
+    if (e0 != cudaSuccess) return fail(cuda_fail(e0, "prep_smooth_kernel"));
+  }
+  if (r > 0) {
+    dim3 g((n + GRAM_T - 1) / GRAM_T, (n + GRAM_T - 1) / GRAM_T);
+    prep_gram_kernel<<<g, 256, 0, st>>>(pw.what, N, K, col_gram, pw.G);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(cuda_fail(e, "prep_gram_kernel"));
+    if (cusolverDnSetStream(h, st) != CUSOLVER_STATUS_SUCCESS ||
+        cusolverDnDsyevd(h, CUSOLVER_EIG_MODE_VECTOR, CUBLAS_FILL_MODE_LOWER, n, pw.G, n, pw.ev,
+                         pw.work, lwork, pw.info) != CUSOLVER_STATUS_SUCCESS) {
+      g_last_error = "cusolverDnDsyevd failed";
+      return fail(SVDQ_ERR_SOLVER);
+    }
+    int info = 0;
+    e = cudaMemcpyAsync(&info, pw.info, sizeof(int), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return fail(cuda_fail(e, "syevd info"));
+    if (info != 0) {
+      g_last_error = "cusolverDnDsyevd info = " + std::to_string(info);
+      return fail(SVDQ_ERR_SOLVER);
+    }
+    const int dot_grid = col_gram ? N : (K + 31) / 32;
+    prep_factor_dot_kernel<<<dot_grid, 256, 0, st>>>(pw.what, N, K, r, col_gram, pw.G, pw.ev, pw.L1f,
+                                                     pw.L2f);
+    prep_factor_direct_kernel<<<nsm * 4, 256, 0, st>>>(N, K, r, col_gram, pw.G, pw.ev, pw.L1f, pw.L2f);
+    prep_sign_kernel<<<r, 256, 0, st>>>(pw.L1f, pw.L2f, N, K, r);
+    prep_round_kernel<<<nsm * 4, 256, 0, st>>>(pw.L1f, pw.L2f, N, K, r, w->L1, w->L2t);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(cuda_fail(e, "prepare factor kernels"));
+  }
+  switch (r_pad_of(r)) {
+    case 0: prep_residual_kernel<0><<<N, 256, 0, st>>>(pw.what, w->L1, w->L2t, N, K, r, w->w_codes, w->w_scales); break;
+    case 16: prep_residual_kernel<16><<<N, 256, 0, st>>>(pw.what, w->L1, w->L2t, N, K, r, w->w_codes, w->w_scales); break;
+    case 32: prep_residual_kernel<32><<<N, 256, 0, st>>>(pw.what, w->L1, w->L2t, N, K, r, w->w_codes, w->w_scales); break;
+    default: prep_residual_kernel<64><<<N, 256, 0, st>>>(pw.what, w->L1, w->L2t, N, K, r, w->w_codes, w->w_scales); break;
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(cuda_fail(e, "prep_residual_kernel"));
+  if (h) cusolverDnDestroy(h);
+  return SVDQ_OK;
+}
+
+svdq_status svdq_quantize_act(const uint16_t* X, int M, const svdq_weight* w, uint8_t* x_codes,
+                              uint8_t* x_scales, uint16_t* D, void* stream) {
+  svdq_status s = check_weight(w);
+  if (s != SVDQ_OK) return s;
+  if (M < 0) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  if (X == nullptr || x_codes == nullptr || x_scales == nullptr || (w->r > 0 && D == nullptr))
+    return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(x_codes) || !aligned16(x_scales) || (w->r > 0 && !aligned16(D)))
+    return SVDQ_ERR_MISALIGNED;
+  return quantize_act_impl(X, M, w, x_codes, x_scales, D, static_cast<cudaStream_t>(stream));
+}
+
+svdq_status svdq_gemm(const uint8_t* x_codes, const uint8_t* x_scales, const uint16_t* D, int M,
+                      const svdq_weight* w, uint16_t* Y, void* stream) {
+  svdq_status s = check_weight(w);
+  if (s != SVDQ_OK) return s;
+  if (M < 0) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  if (x_codes == nullptr || x_scales == nullptr || Y == nullptr || (w->r > 0 && D == nullptr))
+    return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(x_codes) || !aligned16(x_scales) || !aligned16(Y) || (w->r > 0 && !aligned16(D)))
+    return SVDQ_ERR_MISALIGNED;
+  return gemm_impl(x_codes, x_scales, D, M, w, Y, static_cast<cudaStream_t>(stream));
+}
+
+svdq_status svdq_linear_forward(const uint16_t* X, int M, const svdq_weight* w, uint16_t* Y,
+                                void* ws, size_t ws_bytes, void* stream) {
+  svdq_status s = check_weight(w);
+  if (s != SVDQ_OK) return s;
+  if (M < 0) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  if (X == nullptr || Y == nullptr || ws == nullptr) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(Y) || !aligned16(ws)) return SVDQ_ERR_MISALIGNED;
+  if (ws_bytes < act_ws_layout(M, w->K, w->r, nullptr, nullptr)) return SVDQ_ERR_WORKSPACE_TOO_SMALL;
+  ActWs a;
+  act_ws_layout(M, w->K, w->r, static_cast<uint8_t*>(ws), &a);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  s = quantize_act_impl(X, M, w, a.codes, a.scales, a.D, st);
+  if (s != SVDQ_OK) return s;
+  return gemm_impl(a.codes, a.scales, a.D, M, w, Y, st);
+}
+
+svdq_status svdq_linear_forward_host(const uint16_t* X_host, int M, const svdq_weight* w,
+                                     uint16_t* Y_host, uint16_t* X_dev, uint16_t* Y_dev, void* ws,
+                                     size_t ws_bytes, void* stream) {
+  svdq_status s = check_weight(w);
+  if (s != SVDQ_OK) return s;
+  if (M < 0) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  if (X_host == nullptr || Y_host == nullptr) return SVDQ_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  SVDQ_CUDA(cudaMemcpyAsync(X_dev, X_host, static_cast<size_t>(M) * w->K * 2, cudaMemcpyHostToDevice, st));
+  s = svdq_linear_forward(X_dev, M, w, Y_dev, ws, ws_bytes, stream);
+  if (s != SVDQ_OK) return s;
+  SVDQ_CUDA(cudaMemcpyAsync(Y_host, Y_dev, static_cast<size_t>(M) * w->N * 2, cudaMemcpyDeviceToHost, st));
+  return SVDQ_OK;
+}
+
+svdq_status svdq_weight_export(const svdq_weight* w, uint8_t* host_codes, uint8_t* host_scales,
+                               uint16_t* host_L1, uint16_t* host_L2t, float* host_inv_lambda,
+                               void* stream) {
+  svdq_status s = check_weight(w);
+  if (s != SVDQ_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t N = w->N, K = w->K, r = w->r;
+  std::vector<uint8_t> native;
+  if (host_codes) SVDQ_CUDA(cudaMemcpyAsync(host_codes, w->w_codes, N * K / 2, cudaMemcpyDeviceToHost, st));
+  if (host_scales) {
+    native.resize(N * K / 16);
+    SVDQ_CUDA(cudaMemcpyAsync(native.data(), w->w_scales, native.size(), cudaMemcpyDeviceToHost, st));
+  }
+  if (host_L1 && r) SVDQ_CUDA(cudaMemcpyAsync(host_L1, w->L1, K * r * 2, cudaMemcpyDeviceToHost, st));
+  if (host_L2t && r) SVDQ_CUDA(cudaMemcpyAsync(host_L2t, w->L2t, N * r * 2, cudaMemcpyDeviceToHost, st));
+  if (host_inv_lambda)
+    SVDQ_CUDA(cudaMemcpyAsync(host_inv_lambda, w->inv_lambda, K * 4, cudaMemcpyDeviceToHost, st));
+  SVDQ_CUDA(cudaStreamSynchronize(st));
+  if (host_scales) to_logical(native.data(), w->N, w->K, host_scales);
+  return SVDQ_OK;
+}
+
+svdq_status svdq_scales_to_logical(const uint8_t* native, int rows, int K, uint8_t* logical) {
+  if (native == nullptr || logical == nullptr || rows < 0 || K <= 0 || K % 64) return SVDQ_ERR_INVALID_ARG;
+  to_logical(native, rows, K, logical);
+  return SVDQ_OK;
+}
+
+svdq_status svdq_scales_to_native(const uint8_t* logical, int rows, int K, uint8_t* native) {
+  if (native == nullptr || logical == nullptr || rows < 0 || K <= 0 || K % 64) return SVDQ_ERR_INVALID_ARG;
+  const int kb = K / 16;
+  std::memset(native, 0, static_cast<size_t>(m_pad_of(rows)) * kb);
+  for (int i = 0; i < rows; ++i)
+    for (int j = 0; j < kb; ++j) native[sf_offset(i, j, K)] = logical[static_cast<size_t>(i) * kb + j];
+  return SVDQ_OK;
+}
+
+svdq_status svdq_get_device_status(void* stream, uint32_t* detail) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  SVDQ_CUDA(cudaStreamSynchronize(st));
+  unsigned int v = 0;
+  SVDQ_CUDA(cudaMemcpyFromSymbol(&v, g_device_status, sizeof(v)));
+  if (detail) *detail = v;
+  return v ? SVDQ_ERR_TIMEOUT : SVDQ_OK;
+}
+
+svdq_status svdq_clear_device_status(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const unsigned int z = 0;
+  SVDQ_CUDA(cudaMemcpyToSymbolAsync(g_device_status, &z, sizeof(z), 0, cudaMemcpyHostToDevice, st));
+  SVDQ_CUDA(cudaStreamSynchronize(st));
+  return SVDQ_OK;
+}
+
+}  // extern "C"
