@@ -78,45 +78,51 @@ def _profile_traffic(kernel_src: str, name: str):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling during the timed region."""
+    """nvidia-smi clock / throttle sampling (every 100 ms) around the timed region.
+
+    Output goes to a file (nvidia-smi buffers its output when piped) and the
+    sampler is stopped with SIGINT so the last lines are flushed."""
 
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, index: int):
+        import tempfile
         self.index = index
         self.proc = None
-        self.lines = []
+        self.path = tempfile.mktemp(prefix="svdq_clocks_", suffix=".csv")
 
     def __enter__(self):
         try:
+            self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self._t = threading.Thread(target=self._read, daemon=True)
-            self._t.start()
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.fh, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
     def __exit__(self, *a):
+        import signal
         if self.proc is not None:
-            self.proc.terminate()
+            self.proc.send_signal(signal.SIGINT)
             try:
                 self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
+            self.fh.close()
 
     def summary(self):
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
+        try:
+            lines = open(self.path).read().splitlines()
+            os.unlink(self.path)
+        except Exception:
+            lines = []
+        for line in lines:
             f = [x.strip() for x in line.split(",")]
             if len(f) < 9:
                 continue
@@ -135,6 +141,16 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # native (CUDA) arm
 # ---------------------------------------------------------------------------
+
+def _run_for(seconds, flush, step):
+    """Untimed repetitions of the step (with flushes) for about `seconds`."""
+    import torch
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < seconds:
+        for _ in range(10):
+            flush.zero_()
+            step()
+        torch.cuda.synchronize()
 
 def run_native(args):
     import torch
@@ -181,6 +197,8 @@ def run_native(args):
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     with ClockSampler(local) as clk:
+        # the sampler sees >= 0.5 s of this workload before and after the timed steps
+        _run_for(0.5, flush, step)
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
@@ -192,6 +210,7 @@ def run_native(args):
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
+        _run_for(0.5, flush, step)
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = sum(step_ms)
     if world > 1:

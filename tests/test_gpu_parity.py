@@ -4,8 +4,9 @@ Bars ("Parity"):
   * activation and weight NVFP4 codes and E4M3 scales: bit-exact;
   * inv_lambda: bit-exact;
   * D: 1 bf16 ulp + 2^-14 * sum|Xhat L1| (float32 accumulation bound);
-  * Y: max|Y_gpu - Y_oracle| <= 4e-3 rms(Y_oracle), no element beyond 2 bf16 ulps
-    plus that bound; the oracle runs on the library's own exported weight;
+  * Y: every element within 4e-3 rms(Y_oracle) + 2 bf16 ulps of itself; the oracle
+    runs on the library's own exported weight; where the oracle recomputes D
+    itself, D's own tolerance propagated through L2 is added (d_propagated_bound);
   * the rank-r factors: ||L1 L2 - L1o L2o||_F <= 1e-2 ||L1o L2o||_F against the
     oracle's own SVD (bf16 storage of both sides limits this to ~2e-3).
 """
@@ -16,8 +17,8 @@ import w4a4_rank_corrected_act_b200 as svdq
 from oracle import svdq_ref as ref
 from workloads import gen
 
-from gpu_util import (check_d, check_y, dev_f32, dev_u16, dev_u8, empty_u8, stream, to_np_u16,
-                      torch)
+from gpu_util import (check_d, check_y, d_propagated_bound, dev_f32, dev_u16, dev_u8, empty_u8,
+                      stream, to_np_u16, torch)
 
 pytestmark = pytest.mark.gpu
 
@@ -232,7 +233,8 @@ def test_forward_parity(M, K, N, r, with_bias):
     Y = lin.forward(dev_u16(X).view(t.bfloat16))
     t.cuda.synchronize()
     o = ref.linear_forward(X, prep)
-    check_y(to_np_u16(Y.view(t.int16)), o["Y64"], "forward")
+    extra = d_propagated_bound(o["D"], o["D_abs"], exp["L2t"]) if r else None
+    check_y(to_np_u16(Y.view(t.int16)), o["Y64"], "forward", extra=extra)
 
 
 def test_forward_small_workload_end_to_end():
@@ -244,7 +246,8 @@ def test_forward_small_workload_end_to_end():
     lin, exp = _prepare(d["W"], d["lam"], d["bias"], spec.r)
     prep = _oracle_prep_from_export(d["W"], d["lam"], d["bias"], exp, spec.r)
     Y = to_np_u16(lin.forward(dev_u16(d["X"]).view(t.bfloat16)).view(t.int16))
-    check_y(Y, ref.linear_forward(d["X"], prep)["Y64"], "small")
+    o = ref.linear_forward(d["X"], prep)
+    check_y(Y, o["Y64"], "small", extra=d_propagated_bound(o["D"], o["D_abs"], exp["L2t"]))
     own = ref.linear_forward(d["X"], ref.prepare_weight(d["W"], d["lam"], d["bias"], spec.r))["Y64"]
     rms = np.sqrt(np.mean(own ** 2))
     assert np.max(np.abs(ref.bf16_to_f64(Y) - own)) <= 2e-2 * rms * 10  # loose cross-check
