@@ -185,6 +185,35 @@ svdq_status svdq_linear_forward_host(const uint16_t* X_host, int M, const svdq_w
                                      void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Whole layer for callers that cannot allocate device memory.  The pages have
+ * no counterpart of this entry point: it is an interface convenience.
+ *
+ * Some callers cannot call cudaMalloc or receive a workspace: plugin or
+ * extension hosts that hand a layer only its input and output buffers and keep
+ * the device allocator to themselves (an allocation there would bypass the
+ * host's memory pool and its accounting), and latency-critical loops in which
+ * cudaMalloc / cudaFree would synchronise the device.  For them this variant
+ * of svdq_linear_forward takes the activation codes, scales and D from a
+ * fixed scratch array that the library holds in device memory (a file-scope
+ * __device__ array of SVDQ_NOALLOC_SCRATCH_BYTES bytes, resident on every GPU
+ * that loads the library until the process exits).  It calls no allocator.
+ *   X, Y    device, as for svdq_linear_forward (caller-owned).
+ *   Shapes whose workspace (svdq_forward_workspace_bytes) exceeds the scratch
+ *   are rejected with SVDQ_ERR_WORKSPACE_TOO_SMALL and a message in
+ *   svdq_last_error_detail.
+ *   The first call on a device looks up the scratch's device address (with
+ *   that device current) and caches it; make that first call before any
+ *   stream capture.
+ *   Every call shares the one scratch array, which keeps the last call's
+ *   contents: calls whose kernels overlap on the GPU (different streams, or
+ *   several threads) race on it.  Each call overwrites every scratch byte it
+ *   later reads, so nothing needs clearing between calls.
+ * ------------------------------------------------------------------------- */
+#define SVDQ_NOALLOC_SCRATCH_BYTES (64u << 20)
+svdq_status svdq_linear_forward_noalloc(const uint16_t* X, int M, const svdq_weight* w,
+                                        uint16_t* Y, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Test / checkpoint path: copy a prepared weight to host buffers in logical
  * layouts (codes N x K/2, scales N x K/16 row-major, L1 K x r, L2t N x r,
  * inv_lambda K).  Any host pointer may be NULL to skip that field.

@@ -56,6 +56,7 @@ SIGNATURES = {
     "svdq_gemm": (_I, [_P, _P, _P, _I, _WP, _P, _P]),
     "svdq_linear_forward": (_I, [_P, _I, _WP, _P, _P, _SZ, _P]),
     "svdq_linear_forward_host": (_I, [_P, _I, _WP, _P, _P, _P, _P, _SZ, _P]),
+    "svdq_linear_forward_noalloc": (_I, [_P, _I, _WP, _P, _P]),
     "svdq_weight_export": (_I, [_WP, _P, _P, _P, _P, _P, _P]),
     "svdq_scales_to_logical": (_I, [_P, _I, _I, _P]),
     "svdq_scales_to_native": (_I, [_P, _I, _I, _P]),
@@ -163,6 +164,16 @@ def svdq_linear_forward_host(X_host: int, M: int, w: svdq_weight, Y_host: int, X
                              Y_dev: int, ws: int, ws_bytes: int, stream: int) -> None:
     _call("svdq_linear_forward_host", X_host, M, ctypes.byref(w), Y_host, X_dev, Y_dev, ws,
           ws_bytes, stream or None)
+
+
+def svdq_linear_forward_noalloc(X: int, M: int, w: svdq_weight, Y: int, stream: int) -> None:
+    """Whole layer with the library's fixed device scratch (no allocation);
+    for callers that cannot allocate device memory or pass a workspace."""
+    st = lib().svdq_linear_forward_noalloc(X, M, ctypes.byref(w), Y, stream or None)
+    if st == 4:   # shape too large for the fixed scratch: the library says by how much
+        raise SvdqError("svdq_linear_forward_noalloc", st,
+                        lib().svdq_last_error_detail().decode(errors="replace"))
+    _check("svdq_linear_forward_noalloc", st)
 
 
 def svdq_weight_export(w: svdq_weight, host_codes: int, host_scales: int, host_L1: int,

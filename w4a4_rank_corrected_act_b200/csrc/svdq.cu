@@ -377,6 +377,34 @@ void to_logical(const uint8_t* native, int rows, int K, uint8_t* logical) {
       logical[static_cast<size_t>(i) * kb + j] = native[sf_offset(i, j, K)];
 }
 
+// --------------------------------------------------------------------------
+// Fixed device scratch for svdq_linear_forward_noalloc.  Every GPU that loads
+// this library holds it until the process exits.  Host code only ever sees a
+// host-side stand-in for the symbol; its device address comes from
+// cudaGetSymbolAddress, taken once per device with that device current.
+// --------------------------------------------------------------------------
+static __device__ __align__(256) uint8_t g_noalloc_scratch[SVDQ_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[256] = {};
+
+svdq_status noalloc_scratch_address(void** out) {
+  int dev = 0;
+  SVDQ_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 256) {
+    g_last_error = "device ordinal out of range for the no-alloc scratch table";
+    return SVDQ_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    SVDQ_CUDA(cudaGetSymbolAddress(&p, g_noalloc_scratch));
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return SVDQ_OK;
+}
+
 }  // namespace
 
 // ==========================================================================
@@ -588,6 +616,32 @@ svdq_status svdq_linear_forward_host(const uint16_t* X_host, int M, const svdq_w
   if (s != SVDQ_OK) return s;
   SVDQ_CUDA(cudaMemcpyAsync(Y_host, Y_dev, static_cast<size_t>(M) * w->N * 2, cudaMemcpyDeviceToHost, st));
   return SVDQ_OK;
+}
+
+svdq_status svdq_linear_forward_noalloc(const uint16_t* X, int M, const svdq_weight* w, uint16_t* Y,
+                                        void* stream) {
+  svdq_status s = check_weight(w);
+  if (s != SVDQ_OK) return s;
+  if (M < 0) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  if (X == nullptr || Y == nullptr) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(Y)) return SVDQ_ERR_MISALIGNED;
+  const size_t need = act_ws_layout(M, w->K, w->r, nullptr, nullptr);
+  if (need > static_cast<size_t>(SVDQ_NOALLOC_SCRATCH_BYTES)) {
+    g_last_error = "svdq_linear_forward_noalloc: this shape needs " + std::to_string(need) +
+                   " bytes of scratch; the fixed scratch holds " +
+                   std::to_string(static_cast<size_t>(SVDQ_NOALLOC_SCRATCH_BYTES));
+    return SVDQ_ERR_WORKSPACE_TOO_SMALL;
+  }
+  void* scratch = nullptr;
+  s = noalloc_scratch_address(&scratch);
+  if (s != SVDQ_OK) return s;
+  ActWs a;
+  act_ws_layout(M, w->K, w->r, static_cast<uint8_t*>(scratch), &a);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  s = quantize_act_impl(X, M, w, a.codes, a.scales, a.D, st);
+  if (s != SVDQ_OK) return s;
+  return gemm_impl(a.codes, a.scales, a.D, M, w, Y, st);
 }
 
 svdq_status svdq_weight_export(const svdq_weight* w, uint8_t* host_codes, uint8_t* host_scales,
