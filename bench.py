@@ -139,6 +139,26 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
+# multi-rank helpers (one process per GPU; plain replicas, no data collective)
+# ---------------------------------------------------------------------------
+
+def max_over_ranks(x: float, device="cpu") -> float:
+    """Largest value of `x` over all ranks (device time of the slowest rank)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, flops_per_step: float, steps: int, total_ms: float) -> float:
+    """Whole-job TFLOP/s: every rank ran `steps` steps; time = the slowest rank's."""
+    return world * flops_per_step * steps / (total_ms * 1e-3) / 1e12
+
+
+# ---------------------------------------------------------------------------
 # native (CUDA) arm
 # ---------------------------------------------------------------------------
 
@@ -212,17 +232,13 @@ def run_native(args):
             dist.barrier()
         _run_for(0.5, flush, step)
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), device="cuda")
     status = svdq.svdq_get_device_status(sh)
     if status:
         raise SystemExit(f"device status word {status:#x}: a kernel gave up a wait")
 
     flops = 2.0 * M * N * K
-    value = world * flops * args.steps / (total_ms * 1e-3) / 1e12
+    value = job_throughput(world, flops, args.steps, total_ms)
     ms_per_step = total_ms / args.steps
 
     # dominant kernel alone: the FP4 GEMM (svdq_gemm on the act kernel's output),
@@ -285,12 +301,8 @@ def run_native(args):
                                       Y.data_ptr(), ws.data_ptr(), nb, sh)
         e2e_ev[i][1].record(st)
     torch.cuda.synchronize()
-    e2e_ms = sum(s.elapsed_time(e) for s, e in e2e_ev)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e = {"value": round(world * flops * args.steps / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
+    e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in e2e_ev), device="cuda")
+    e2e = {"value": round(job_throughput(world, flops, args.steps, e2e_ms), 2), "unit": UNIT,
            "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2,
            "ms_per_step": round(e2e_ms / args.steps, 4)}
 

@@ -77,6 +77,11 @@ typedef enum svdq_status {
  *              (rb * K/64 + kb) * 512, and inside a tile, row i and scale j at
  *              (i % 32) * 16 + (i / 32) * 4 + j.  Size N * K / 16 bytes.
  *   L1         K x r bf16, L1 = U_r diag(sigma_r) of the smoothed weight.
+ *   L1f        the same K x r values in the B-fragment order of the warp-level
+ *              bf16 MMA m16n8k16 (read by the activation kernel): for k-step
+ *              g = k/16 and column tile t = j/8, the 32 lanes' fragments follow
+ *              each other; 32-bit word ((g * r/8 + t) * 32 + lane) * 2 + h holds
+ *              L1[16g + 2(lane%4) + 8h + {0 (low half), 1}][8t + lane/4].
  *   L2t        N x r bf16, L2^T = V_r.
  *   inv_lambda K float32, f32(1 / lambda).
  *   bias       N bf16, or NULL when has_bias == 0.
@@ -87,6 +92,7 @@ typedef struct svdq_weight {
   uint8_t* w_codes;
   uint8_t* w_scales;
   uint16_t* L1;
+  uint16_t* L1f;
   uint16_t* L2t;
   float* inv_lambda;
   uint16_t* bias;

@@ -46,7 +46,8 @@ def test_sizes():
     al = lambda x: (x + 255) // 256 * 256                              # noqa: E731
     M, N, K, r = 4608, 9216, 3072, 32
     assert svdq.svdq_forward_workspace_bytes(M, N, K, r) == al(M * K // 2) + al(M * K // 16) + al(M * r * 2)
-    wb = al(N * K // 2) + al(N * K // 16) + al(K * r * 2) + al(N * r * 2) + al(K * 4) + al(N * 2)
+    wb = (al(N * K // 2) + al(N * K // 16) + al(K * r * 2) + al(K * r * 2) + al(N * r * 2)
+          + al(K * 4) + al(N * 2))
     assert svdq.svdq_weight_bytes(N, K, r, 1) == wb
     assert svdq.svdq_weight_bytes(N, K, r, 0) == wb - al(N * 2)
 
@@ -64,7 +65,7 @@ def test_weight_bind_carves_aligned_fields():
     nbytes = svdq.svdq_weight_bytes(N, K, r, 1)
     base = 0x7F0000000000                   # never dereferenced: bind is pointer arithmetic
     w = svdq.svdq_weight_bind(base, nbytes, N, K, r, 1)
-    fields = [w.w_codes, w.w_scales, w.L1, w.L2t, w.inv_lambda, w.bias]
+    fields = [w.w_codes, w.w_scales, w.L1, w.L1f, w.L2t, w.inv_lambda, w.bias]
     assert all(f % 256 == 0 for f in fields)
     assert fields == sorted(fields) and fields[0] == base
     assert w.bias + N * 2 <= base + nbytes

@@ -56,7 +56,23 @@ def _weight_with(K, N, r, inv_lambda, L1=None, has_bias=False):
     put(w.inv_lambda, inv_lambda.astype(np.float32))
     if r:
         put(w.L1, L1.astype(np.uint16))
+        put(w.L1f, l1_fragment_order(L1.astype(np.uint16)))
     return w, buf
+
+
+def l1_fragment_order(L1):
+    """L1 (K x r) in the B-fragment order documented in include/svdq.h: 32-bit word
+    ((g * r/8 + t) * 32 + lane) * 2 + h holds L1[16g + 2(lane%4) + 8h + {0, 1}][8t + lane/4]."""
+    K, r = L1.shape
+    out = np.zeros(K * r, np.uint16)
+    for k in range(K):
+        g, kk = divmod(k, 16)
+        for j in range(r):
+            t, jj = divmod(j, 8)
+            lane = jj * 4 + (kk % 8) // 2
+            word = ((g * (r // 8) + t) * 32 + lane) * 2 + kk // 8
+            out[word * 2 + (k & 1)] = L1[k, j]
+    return out
 
 
 def _run_act(X, inv, L1, N=128):

@@ -34,7 +34,7 @@ class svdq_weight(ctypes.Structure):
     _fields_ = [
         ("N", ctypes.c_int32), ("K", ctypes.c_int32), ("r", ctypes.c_int32),
         ("has_bias", ctypes.c_int32),
-        ("w_codes", _P), ("w_scales", _P), ("L1", _P), ("L2t", _P),
+        ("w_codes", _P), ("w_scales", _P), ("L1", _P), ("L1f", _P), ("L2t", _P),
         ("inv_lambda", _P), ("bias", _P),
     ]
 

@@ -9,14 +9,20 @@
 // Blackwell/B200 precision (chaosnode.de "Nunchaku Lite", section
 // "Hardware-Support").
 //
-// Per 128 x BN output tile, one fp32 accumulator lives in tensor memory:
+// Per 128 x BN output tile, an fp32 accumulator lives in tensor memory:
 //   1. the low-rank term: R_PAD/16 bf16 MMAs (kind::f16, K = 16) of the D tile
 //      (128 x r) against the L2^T tile (BN x r) initialise the accumulator;
 //   2. K/64 block-scaled MMAs (kind::mxf4nvf4, K = 64, one UE4M3 scale per 16)
 //      accumulate the 4-bit product; scales are copied shared -> tensor memory
 //      with tcgen05.cp right before the MMAs that read them;
 //   3. the epilogue reads the accumulator with tcgen05.ld, adds the bias,
-//      rounds to bf16 and stores Y.
+//      rounds to bf16, stages 32 x 32 pieces in shared memory and stores Y
+//      with TMA.
+// Two accumulator buffers alternate between tiles so the epilogue of tile t
+// overlaps the MMAs of tile t+1.  With BN = 256 they cannot both fit next to
+// the scale columns (2 x 256 + 64 > 512), so buffer 1 starts at column 192 and
+// shares 64 columns with buffer 0; the epilogue reads those shared columns of a
+// tile first and releases them before draining the rest.
 // Warp roles (256 threads): warp 0 issues TMA / bulk copies into a STAGES-deep
 // shared-memory ring, warp 1 issues the MMAs (one thread), warp 2 owns the
 // tensor-memory allocation, warps 4-7 run the epilogue (warp w reads lanes
@@ -33,12 +39,12 @@ constexpr int GEMM_BK = 256;                 // fp4 elements per stage = 128 byt
 constexpr int GEMM_THREADS = 256;
 constexpr uint32_t GEMM_A_TILE = GEMM_BM * 128;   // 16 KB
 constexpr uint32_t GEMM_SFA_TILE = 4 * 512;       // 4 scale tiles (4 x 64 K) for 128 rows
+constexpr uint32_t GEMM_STAGE_OUT = 32 * 64;      // per epilogue warp: 32 rows x 32 bf16
 
 struct GemmParams {
   const uint8_t* x_scales;
   const uint8_t* w_scales;
   const uint16_t* bias;
-  uint16_t* Y;
   int M, N, K, r;
   int m_tiles, n_tiles, num_tiles, kblocks;
 };
@@ -49,12 +55,19 @@ struct GemmCfg {
   static constexpr uint32_t kSFBTile = (BN / 128) * GEMM_SFA_TILE;
   static constexpr uint32_t kStage = GEMM_A_TILE + kBTile + GEMM_SFA_TILE + kSFBTile;
   static constexpr int kStages = (BN == 256 ? 4 : 6);
-  static constexpr uint32_t kSfColsPerStage = 16 + BN / 8;   // SFA 4x4 + SFB 4x(BN/32)
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kBarBytes = (2 * kStages + 3) * 8 + 16;
-  static constexpr uint32_t kSmemBytes = kStages * kStage + kBarBytes + 1024;
-  static_assert(BN + kStages * kSfColsPerStage <= kTmemCols, "tensor memory budget");
+  // tensor-memory columns: scales in the top 64, accumulator buffers below
+  static constexpr uint32_t kSfaCol = 448;               // 4 k-blocks x 4 columns
+  static constexpr uint32_t kSfbCol = 464;               // 4 k-blocks x BN/32 columns
+  static constexpr uint32_t kAcc1Col = (BN == 256 ? 192 : 128);
+  static constexpr int kOverlapChunks = (BN == 256 ? (256 - 192) / 32 : 0);
+  static constexpr uint32_t kOutBytes = 4 * GEMM_STAGE_OUT;   // epilogue staging, 4 warps
+  static constexpr uint32_t kBarBytes = (2 * kStages + 4) * 8 + 16;
+  static constexpr uint32_t kSmemBytes = kStages * kStage + kOutBytes + kBarBytes + 1024;
+  static_assert(kSfbCol + 4 * (BN / 32) <= kTmemCols, "scale columns");
+  static_assert(kAcc1Col + BN <= kSfaCol, "accumulator buffer 1");
   static_assert(kStage % 1024 == 0, "stage alignment");
+  static_assert(kSmemBytes <= 232448, "shared memory");
 };
 
 // Instruction descriptors (tcgen05.mma, 32-bit):
@@ -77,18 +90,20 @@ template <int BN, int R_PAD>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     fp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                     const __grid_constant__ CUtensorMap tm_d, const __grid_constant__ CUtensorMap tm_l2,
-                    const GemmParams p) {
+                    const __grid_constant__ CUtensorMap tm_y, const GemmParams p) {
   using Cfg = GemmCfg<BN>;
   constexpr int S = Cfg::kStages;
   constexpr uint32_t kLRLayout = (R_PAD == 64 ? LAYOUT_SW128 : R_PAD == 32 ? LAYOUT_SW64 : LAYOUT_SW32);
   constexpr uint32_t kLRSbo = 8 * R_PAD * 2;
+  constexpr int kChunks = BN / 32;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * Cfg::kStage);
-  // bars[0..S): full, [S..2S): empty, 2S: tmem_full, 2S+1: tmem_empty, 2S+2: drain
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 3);
+  uint8_t* out_stage = smem + S * Cfg::kStage;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(out_stage + Cfg::kOutBytes);
+  // bars[0..S) full, [S..2S) empty, 2S/2S+1 tmem_full[2], 2S+2 tmem_free, 2S+3 drain
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -101,17 +116,18 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   };
   auto full_bar = [&](int s) { return smem_u32(bars + s); };
   auto empty_bar = [&](int s) { return smem_u32(bars + S + s); };
-  const uint32_t tmem_full = smem_u32(bars + 2 * S);
-  const uint32_t tmem_empty = smem_u32(bars + 2 * S + 1);
-  const uint32_t drain_bar = smem_u32(bars + 2 * S + 2);
+  auto tmem_full = [&](int b) { return smem_u32(bars + 2 * S + b); };
+  const uint32_t tmem_free = smem_u32(bars + 2 * S + 2);
+  const uint32_t drain_bar = smem_u32(bars + 2 * S + 3);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), 1);
     }
-    mbar_init(tmem_full, 1);
-    mbar_init(tmem_empty, 128);
+    mbar_init(tmem_full(0), 1);
+    mbar_init(tmem_full(1), 1);
+    mbar_init(tmem_free, 128);
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -139,7 +155,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       }
       int stage = 0;
       uint32_t phase = 0;
-      int issued = 0;
       int8_t fill_parity[S];
       for (int s = 0; s < S; ++s) fill_parity[s] = -1;
       const uint32_t tx_main = GEMM_A_TILE + Cfg::kBTile + GEMM_SFA_TILE + Cfg::kSFBTile;
@@ -154,7 +169,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           tma_load_2d(stage_a(stage), &tm_d, full_bar(stage), 0, m0);
           tma_load_2d(stage_b(stage), &tm_l2, full_bar(stage), 0, n0);
           fill_parity[stage] = static_cast<int8_t>(phase);
-          ++issued;
           if (++stage == S) { stage = 0; phase ^= 1; }
         }
         for (int kb = 0; kb < kb_per_tile; ++kb) {
@@ -171,16 +185,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                       p.w_scales + (static_cast<size_t>(n0 / 128 + g) * k_tiles64 + kb * 4) * 512,
                       GEMM_SFA_TILE, full_bar(stage));
           fill_parity[stage] = static_cast<int8_t>(phase);
-          ++issued;
           if (++stage == S) { stage = 0; phase ^= 1; }
         }
       }
       if (*abort_flag) {
         for (int s = 0; s < S; ++s)
-          if (fill_parity[s] >= 0)
-            mbar_wait_drain(full_bar(s), static_cast<uint32_t>(fill_parity[s]));
+          if (fill_parity[s] >= 0) mbar_wait_drain(full_bar(s), static_cast<uint32_t>(fill_parity[s]));
       }
-      (void)issued;
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -188,11 +199,21 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       const uint32_t idf = idesc_nvfp4(GEMM_BM, BN);
       const uint32_t idb = idesc_bf16(GEMM_BM, BN);
       int stage = 0;
-      uint32_t phase = 0, acc_phase = 0;
+      uint32_t phase = 0;
       bool ok = true;
       bool any_issued = false;
-      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
-        if (!mbar_wait(tmem_empty, acc_phase ^ 1, abort_flag, KID_GEMM, 4)) { ok = false; break; }
+      int local = 0;   // tiles issued by this CTA
+      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x, ++local) {
+        const int buf = local & 1;
+        const uint32_t acc = tmem_base + (buf ? Cfg::kAcc1Col : 0u);
+        // the epilogue has drained the previous tile's shared columns (and so
+        // everything of the tile before it, which used this buffer)
+        if (local > 0) {
+          if (!mbar_wait(tmem_free, static_cast<uint32_t>(local - 1) & 1u, abort_flag, KID_GEMM, 4)) {
+            ok = false;
+            break;
+          }
+        }
         tc_fence_after();
         uint32_t accumulate = 0;
         if (R_PAD > 0) {
@@ -202,7 +223,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           const uint64_t bd = make_smem_desc(stage_b(stage), kLRLayout, kLRSbo, 0);
 #pragma unroll
           for (int kk = 0; kk < R_PAD / 16; ++kk) {
-            tc_mma_bf16(tmem_base, ad + 2 * kk, bd + 2 * kk, idb, accumulate);
+            tc_mma_bf16(acc, ad + 2 * kk, bd + 2 * kk, idb, accumulate);
             accumulate = 1;
           }
           tc_commit(empty_bar(stage));
@@ -212,25 +233,25 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         for (int kb = 0; kb < kb_per_tile; ++kb) {
           if (!mbar_wait(full_bar(stage), phase, abort_flag, KID_GEMM, 6)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sf_cols = BN + stage * Cfg::kSfColsPerStage;
-          // scale factors: shared -> tensor memory (32 rows x 16 B per copy)
+          // scale factors: shared -> tensor memory (32 rows x 16 B per copy); the
+          // region is reused by every stage (tcgen05 ops of a thread run in order)
 #pragma unroll
           for (int i = 0; i < 4; ++i)
-            tc_cp_32x128b_warpx4(tmem_base + sf_cols + 4 * i,
+            tc_cp_32x128b_warpx4(tmem_base + Cfg::kSfaCol + 4 * i,
                                  make_smem_desc(stage_sfa(stage) + i * 512, LAYOUT_NONE, 128, 0));
 #pragma unroll
           for (int i = 0; i < 4; ++i)
 #pragma unroll
             for (int g = 0; g < BN / 128; ++g)
               tc_cp_32x128b_warpx4(
-                  tmem_base + sf_cols + 16 + i * (BN / 32) + 4 * g,
+                  tmem_base + Cfg::kSfbCol + i * (BN / 32) + 4 * g,
                   make_smem_desc(stage_sfb(stage) + (g * 4 + i) * 512, LAYOUT_NONE, 128, 0));
           const uint64_t ad = make_smem_desc(stage_a(stage), LAYOUT_SW128, 1024, 0);
           const uint64_t bd = make_smem_desc(stage_b(stage), LAYOUT_SW128, 1024, 0);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            tc_mma_nvfp4(tmem_base, ad + 2 * i, bd + 2 * i, idf, tmem_base + sf_cols + 4 * i,
-                         tmem_base + sf_cols + 16 + i * (BN / 32), accumulate);
+            tc_mma_nvfp4(acc, ad + 2 * i, bd + 2 * i, idf, tmem_base + Cfg::kSfaCol + 4 * i,
+                         tmem_base + Cfg::kSfbCol + i * (BN / 32), accumulate);
             accumulate = 1;
           }
           tc_commit(empty_bar(stage));
@@ -238,8 +259,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           if (++stage == S) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
-        tc_commit(tmem_full);
-        acc_phase ^= 1;
+        tc_commit(tmem_full(buf));
       }
       if (*abort_flag && any_issued) {
         // make sure no MMA still writes tensor memory before it is freed
@@ -250,19 +270,30 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   } else if (warp >= 4) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
-    uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
+    uint8_t* stg = out_stage + q * GEMM_STAGE_OUT;
+    const uint32_t stg_u = smem_u32(stg);
+    const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+    int local = 0;
+    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++local) {
       const int mb = t % p.m_tiles, nb = t / p.m_tiles;
       const int m0 = mb * GEMM_BM, n0 = nb * BN;
-      if (!mbar_wait(tmem_full, acc_phase, abort_flag, KID_GEMM, 8)) break;
+      const int buf = local & 1;
+      const uint32_t acc = tmem_base + (buf ? Cfg::kAcc1Col : 0u);
+      if (!mbar_wait(tmem_full(buf), static_cast<uint32_t>(local >> 1) & 1u, abort_flag, KID_GEMM, 8))
+        break;
       tc_fence_after();
-      const int row = m0 + q * 32 + lane;
-      uint16_t* yrow = p.Y + static_cast<size_t>(row) * p.N + n0;
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int i = 0; i < kChunks; ++i) {
+        // buffer 0 shares its top chunks with buffer 1, buffer 1 its bottom
+        // chunks with buffer 0: those come first, then the columns are released
+        const int c = buf ? i : (i + kChunks - Cfg::kOverlapChunks) % kChunks;
         uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + c * 32, v);
+        tmem_ld_32x32b_x32(acc + lane_addr + c * 32, v);
         tmem_ld_wait();
+        if (i + 1 == Cfg::kOverlapChunks || (Cfg::kOverlapChunks == 0 && i == 0)) {
+          tc_fence_before();
+          mbar_arrive(tmem_free);
+        }
         float f[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[j]);
@@ -279,23 +310,29 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             }
           }
         }
-        if (row < p.M) {
-          uint4* dst = reinterpret_cast<uint4*>(yrow + c * 32);
+        // the previous store of this warp must have finished reading the staging
+        if (lane == 0) bulk_wait_group_read<0>();
+        __syncwarp();
+        // row `lane` of the 32 x 32 piece, 64-byte swizzled (the TMA store's layout)
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            uint4 o;
-            o.x = pack_bf16x2(f[u * 8 + 0], f[u * 8 + 1]);
-            o.y = pack_bf16x2(f[u * 8 + 2], f[u * 8 + 3]);
-            o.z = pack_bf16x2(f[u * 8 + 4], f[u * 8 + 5]);
-            o.w = pack_bf16x2(f[u * 8 + 6], f[u * 8 + 7]);
-            dst[u] = o;
-          }
+        for (int u = 0; u < 4; ++u) {
+          uint4 o;
+          o.x = pack_bf16x2(f[u * 8 + 0], f[u * 8 + 1]);
+          o.y = pack_bf16x2(f[u * 8 + 2], f[u * 8 + 3]);
+          o.z = pack_bf16x2(f[u * 8 + 4], f[u * 8 + 5]);
+          o.w = pack_bf16x2(f[u * 8 + 6], f[u * 8 + 7]);
+          *reinterpret_cast<uint4*>(stg + swz(lane * 64 + u * 16, 2)) = o;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tm_y, stg_u, n0 + c * 32, m0 + q * 32);
+          bulk_commit_group();
         }
       }
-      tc_fence_before();
-      mbar_arrive(tmem_empty);
-      acc_phase ^= 1;
     }
+    if (lane == 0) bulk_wait_group_all();
+    __syncwarp();
   }
 
   tc_fence_before();

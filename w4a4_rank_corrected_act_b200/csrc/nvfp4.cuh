@@ -49,10 +49,28 @@ __device__ __forceinline__ uint32_t e2m1x8_magnitudes(const float (&a)[8]) {
   return out;
 }
 
+// E2M1 magnitude codes of 8 non-negative float32 bit patterns.
+__device__ __forceinline__ uint32_t e2m1x8_of_bits(const uint32_t (&b)[8]) {
+  const float a[8] = {__uint_as_float(b[0]), __uint_as_float(b[1]), __uint_as_float(b[2]),
+                      __uint_as_float(b[3]), __uint_as_float(b[4]), __uint_as_float(b[5]),
+                      __uint_as_float(b[6]), __uint_as_float(b[7])};
+  return e2m1x8_magnitudes(a);
+}
+
 // Quantise 8 consecutive values forming one half of a 16-element block; the
 // other half lives on lane (laneid ^ 1).  Must be called by all 32 lanes of
 // the warp.  Returns the 8 packed codes; `scale_code` receives the block's
 // E4M3 code (identical on both lanes of the pair).
+//
+// The codes are E2M1_rn(RN(v_i / s)) exactly, without one IEEE division per
+// element: q_i = RN(v_i * RN(1/s)) differs from v_i / s by at most
+// (2^-23 + 2^-48) |v_i / s|, i.e. by less than 2 ulps of q_i, and RN(v_i / s)
+// lies within half an ulp of v_i / s; so RN(v_i / s) is inside [lo, hi], the
+// float32 values 4 representable steps below and above |q_i| (4 steps span at
+// least 2 ulps even across a binade boundary).  E2M1 rounding is monotone, so
+// when lo and hi get the same code every value in between does too, and that
+// code is the answer.  Otherwise (|q_i| within a few ulps of a rounding
+// threshold, exact ties included) the block takes the IEEE division.
 __device__ __forceinline__ uint32_t nvfp4_quant_half_block(const float (&v)[8],
                                                           uint32_t& scale_code) {
   float am = 0.0f;
@@ -61,15 +79,25 @@ __device__ __forceinline__ uint32_t nvfp4_quant_half_block(const float (&v)[8],
   am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
   const uint32_t sc = e4m3_rn_satfinite(__fdiv_rn(am, 6.0f));
   const float s = e4m3_to_f32(sc);
-  float mag[8];
+  scale_code = sc;
   uint32_t signs = 0;
 #pragma unroll
+  for (int i = 0; i < 8; ++i) signs |= (__float_as_uint(v[i]) >> 31) << (4 * i + 3);
+  if (s == 0.0f) return signs;                 // every |v_i| / s taken as +-0
+  const float inv_s = __frcp_rn(s);
+  uint32_t lo[8], hi[8];
+#pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const float q = (s == 0.0f) ? 0.0f : __fdiv_rn(v[i], s);
-    mag[i] = fabsf(q);
-    signs |= (__float_as_uint(v[i]) >> 31) << (4 * i + 3);
+    const uint32_t m = __float_as_uint(fabsf(__fmul_rn(v[i], inv_s)));
+    lo[i] = (m > 4u ? m : 4u) - 4u;
+    hi[i] = m + 4u;
   }
-  scale_code = sc;
+  const uint32_t clo = e2m1x8_of_bits(lo);
+  const uint32_t chi = e2m1x8_of_bits(hi);
+  if (clo == chi) return clo | signs;
+  float mag[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) mag[i] = fabsf(__fdiv_rn(v[i], s));
   return e2m1x8_magnitudes(mag) | signs;
 }
 

@@ -71,10 +71,11 @@ svdq_status check_weight(const svdq_weight* w) {
   if (s != SVDQ_OK) return s;
   if (w->w_codes == nullptr || w->w_scales == nullptr || w->inv_lambda == nullptr)
     return SVDQ_ERR_INVALID_ARG;
-  if (w->r > 0 && (w->L1 == nullptr || w->L2t == nullptr)) return SVDQ_ERR_INVALID_ARG;
+  if (w->r > 0 && (w->L1 == nullptr || w->L1f == nullptr || w->L2t == nullptr))
+    return SVDQ_ERR_INVALID_ARG;
   if (w->has_bias && w->bias == nullptr) return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(w->w_codes) || !aligned16(w->w_scales) || !aligned16(w->inv_lambda) ||
-      (w->r > 0 && (!aligned16(w->L1) || !aligned16(w->L2t))) ||
+      (w->r > 0 && (!aligned16(w->L1) || !aligned16(w->L1f) || !aligned16(w->L2t))) ||
       (w->has_bias && !aligned16(w->bias)))
     return SVDQ_ERR_MISALIGNED;
   return SVDQ_OK;
@@ -142,25 +143,25 @@ int num_sms() {
 // Launchers
 // --------------------------------------------------------------------------
 template <int R_PAD>
-svdq_status launch_act(const CUtensorMap& tx, const CUtensorMap& tl1, const ActParams& p,
-                       cudaStream_t st) {
-  const uint32_t smem = ActSmem<R_PAD>::bytes(p.stages);
+svdq_status launch_act(const CUtensorMap& tx, const ActParams& p, cudaStream_t st) {
+  constexpr uint32_t smem = ActSmem<R_PAD>::kBytes;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [&] {
     attr_err = cudaFuncSetAttribute(act_quant_kernel<R_PAD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    227 * 1024);
+                                    smem);
   });
   if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(act)");
-  const int grid = p.M_pad / ACT_BM;
-  act_quant_kernel<R_PAD><<<grid, ACT_THREADS, smem, st>>>(tx, tl1, p);
+  const int grid = p.M_pad / ACT_ROWS;
+  act_quant_kernel<R_PAD><<<grid, ACT_THREADS, smem, st>>>(tx, p);
   SVDQ_CHECK_LAUNCH("act_quant_kernel");
   return SVDQ_OK;
 }
 
 template <int BN, int R_PAD>
 svdq_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
-                        const CUtensorMap& tl2, const GemmParams& p, cudaStream_t st) {
+                        const CUtensorMap& tl2, const CUtensorMap& ty, const GemmParams& p,
+                        cudaStream_t st) {
   using Cfg = GemmCfg<BN>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
@@ -170,53 +171,34 @@ svdq_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUte
   });
   if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(gemm)");
   const int grid = std::min(p.num_tiles, num_sms());
-  fp4_gemm_kernel<BN, R_PAD><<<grid, GEMM_THREADS, Cfg::kSmemBytes, st>>>(ta, tb, td, tl2, p);
+  fp4_gemm_kernel<BN, R_PAD><<<grid, GEMM_THREADS, Cfg::kSmemBytes, st>>>(ta, tb, td, tl2, ty, p);
   SVDQ_CHECK_LAUNCH("fp4_gemm_kernel");
   return SVDQ_OK;
 }
 
 template <int BN>
 svdq_status dispatch_gemm_r(int r_pad, const CUtensorMap& ta, const CUtensorMap& tb,
-                            const CUtensorMap& td, const CUtensorMap& tl2, const GemmParams& p,
-                            cudaStream_t st) {
+                            const CUtensorMap& td, const CUtensorMap& tl2, const CUtensorMap& ty,
+                            const GemmParams& p, cudaStream_t st) {
   switch (r_pad) {
-    case 0: return launch_gemm<BN, 0>(ta, tb, td, tl2, p, st);
-    case 16: return launch_gemm<BN, 16>(ta, tb, td, tl2, p, st);
-    case 32: return launch_gemm<BN, 32>(ta, tb, td, tl2, p, st);
-    default: return launch_gemm<BN, 64>(ta, tb, td, tl2, p, st);
+    case 0: return launch_gemm<BN, 0>(ta, tb, td, tl2, ty, p, st);
+    case 16: return launch_gemm<BN, 16>(ta, tb, td, tl2, ty, p, st);
+    case 32: return launch_gemm<BN, 32>(ta, tb, td, tl2, ty, p, st);
+    default: return launch_gemm<BN, 64>(ta, tb, td, tl2, ty, p, st);
   }
-}
-
-int act_stages(int r_pad) {
-  // as many 16 KB + L1-slice stages as fit next to the reduction buffer (max 4)
-  const uint32_t budget = 227 * 1024;
-  for (int s = 4; s >= 2; --s) {
-    uint32_t b = 0;
-    switch (r_pad) {
-      case 0: b = ActSmem<0>::bytes(s); break;
-      case 16: b = ActSmem<16>::bytes(s); break;
-      case 32: b = ActSmem<32>::bytes(s); break;
-      default: b = ActSmem<64>::bytes(s); break;
-    }
-    if (b <= budget) return s;
-  }
-  return 2;
 }
 
 svdq_status quantize_act_impl(const uint16_t* X, int M, const svdq_weight* w, uint8_t* x_codes,
                               uint8_t* x_scales, uint16_t* D, cudaStream_t st) {
   const int K = w->K, r = w->r, rp = r_pad_of(r);
-  CUtensorMap tx{}, tl1{};
+  CUtensorMap tx{};
   svdq_status s = make_tmap(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M,
-                            static_cast<uint64_t>(K) * 2, 64, ACT_BM, CU_TENSOR_MAP_SWIZZLE_128B);
+                            static_cast<uint64_t>(K) * 2, ACT_SUB, ACT_ROWS,
+                            CU_TENSOR_MAP_SWIZZLE_128B);
   if (s != SVDQ_OK) return s;
-  if (r > 0) {
-    s = make_tmap(&tl1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->L1, r, K, static_cast<uint64_t>(r) * 2,
-                  rp, ACT_KC, lr_swizzle(rp));
-    if (s != SVDQ_OK) return s;
-  }
   ActParams p;
   p.inv_lambda = w->inv_lambda;
+  p.L1f = reinterpret_cast<const uint32_t*>(w->L1f);
   p.x_codes = x_codes;
   p.x_scales = x_scales;
   p.D = D;
@@ -224,12 +206,11 @@ svdq_status quantize_act_impl(const uint16_t* X, int M, const svdq_weight* w, ui
   p.K = K;
   p.r = r;
   p.M_pad = m_pad_of(M);
-  p.stages = act_stages(rp);
   switch (rp) {
-    case 0: return launch_act<0>(tx, tl1, p, st);
-    case 16: return launch_act<16>(tx, tl1, p, st);
-    case 32: return launch_act<32>(tx, tl1, p, st);
-    default: return launch_act<64>(tx, tl1, p, st);
+    case 0: return launch_act<0>(tx, p, st);
+    case 16: return launch_act<16>(tx, p, st);
+    case 32: return launch_act<32>(tx, p, st);
+    default: return launch_act<64>(tx, p, st);
   }
 }
 
@@ -244,12 +225,16 @@ svdq_status gemm_impl(const uint8_t* x_codes, const uint8_t* x_scales, const uin
     const int v = std::atoi(e);
     if (v == 128 || (v == 256 && N % 256 == 0)) BN = v;
   }
-  CUtensorMap ta{}, tb{}, td{}, tl2{};
+  CUtensorMap ta{}, tb{}, td{}, tl2{}, ty{};
   svdq_status s = make_tmap(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, x_codes, K / 2, M, K / 2, 128,
                             GEMM_BM, CU_TENSOR_MAP_SWIZZLE_128B);
   if (s != SVDQ_OK) return s;
   s = make_tmap(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->w_codes, K / 2, N, K / 2, 128, BN,
                 CU_TENSOR_MAP_SWIZZLE_128B);
+  if (s != SVDQ_OK) return s;
+  // Y is stored in 32 x 32 pieces through 64-byte-swizzled staging buffers
+  s = make_tmap(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, N, M, static_cast<uint64_t>(N) * 2, 32, 32,
+                CU_TENSOR_MAP_SWIZZLE_64B);
   if (s != SVDQ_OK) return s;
   if (r > 0) {
     s = make_tmap(&td, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, D, r, M, static_cast<uint64_t>(r) * 2, rp,
@@ -263,7 +248,6 @@ svdq_status gemm_impl(const uint8_t* x_codes, const uint8_t* x_scales, const uin
   p.x_scales = x_scales;
   p.w_scales = w->w_scales;
   p.bias = w->has_bias ? w->bias : nullptr;
-  p.Y = Y;
   p.M = M;
   p.N = N;
   p.K = K;
@@ -272,8 +256,8 @@ svdq_status gemm_impl(const uint8_t* x_codes, const uint8_t* x_scales, const uin
   p.n_tiles = N / BN;
   p.num_tiles = p.m_tiles * p.n_tiles;
   p.kblocks = K / GEMM_BK;
-  return BN == 256 ? dispatch_gemm_r<256>(rp, ta, tb, td, tl2, p, st)
-                   : dispatch_gemm_r<128>(rp, ta, tb, td, tl2, p, st);
+  return BN == 256 ? dispatch_gemm_r<256>(rp, ta, tb, td, tl2, ty, p, st)
+                   : dispatch_gemm_r<128>(rp, ta, tb, td, tl2, ty, p, st);
 }
 
 struct ActWs {
@@ -305,6 +289,7 @@ size_t weight_layout(int N, int K, int r, int has_bias, uint8_t* base, svdq_weig
   uint8_t* codes = take(static_cast<size_t>(N) * (K / 2));
   uint8_t* scales = take(static_cast<size_t>(N) * (K / 16));
   uint8_t* l1 = take(static_cast<size_t>(K) * r * 2);
+  uint8_t* l1f = take(static_cast<size_t>(K) * r * 2);
   uint8_t* l2t = take(static_cast<size_t>(N) * r * 2);
   uint8_t* inv = take(static_cast<size_t>(K) * 4);
   uint8_t* bias = has_bias ? take(static_cast<size_t>(N) * 2) : nullptr;
@@ -316,6 +301,7 @@ size_t weight_layout(int N, int K, int r, int has_bias, uint8_t* base, svdq_weig
     out->w_codes = codes;
     out->w_scales = scales;
     out->L1 = r > 0 ? reinterpret_cast<uint16_t*>(l1) : nullptr;
+    out->L1f = r > 0 ? reinterpret_cast<uint16_t*>(l1f) : nullptr;
     out->L2t = r > 0 ? reinterpret_cast<uint16_t*>(l2t) : nullptr;
     out->inv_lambda = reinterpret_cast<float*>(inv);
     out->bias = reinterpret_cast<uint16_t*>(bias);
@@ -544,6 +530,7 @@ svdq_status svdq_prepare_weight(const uint16_t* W, const float* lambda, const ui
     prep_factor_direct_kernel<<<nsm * 4, 256, 0, st>>>(N, K, r, col_gram, pw.G, pw.ev, pw.L1f, pw.L2f);
     prep_sign_kernel<<<r, 256, 0, st>>>(pw.L1f, pw.L2f, N, K, r);
     prep_round_kernel<<<nsm * 4, 256, 0, st>>>(pw.L1f, pw.L2f, N, K, r, w->L1, w->L2t);
+    l1_fragment_kernel<<<nsm * 2, 256, 0, st>>>(w->L1, K, r, w->L1f);
     e = cudaGetLastError();
     if (e != cudaSuccess) return fail(cuda_fail(e, "prepare factor kernels"));
   }
