@@ -42,7 +42,9 @@
  *     A CUDA launch/runtime failure is SVDQ_ERR_CUDA (its text is kept in a
  *     thread-local string, see svdq_last_error_detail).
  *   - The library is stateless apart from a per-device status word that
- *     kernels set when a bounded wait times out (svdq_get_device_status).
+ *     kernels set when a bounded wait times out (svdq_get_device_status):
+ *     bit 0 = timeout, bits 8-15 = kernel (1 activation, 2 GEMM, 3 prepare,
+ *     4 self-test), bits 16-23 = wait site.  Every wait gives up after 1 s.
  */
 #ifndef SVDQ_H_
 #define SVDQ_H_
@@ -167,9 +169,10 @@ svdq_status svdq_quantize_act(const uint16_t* X, int M, const svdq_weight* w, ui
  * Block-scaled FP4 GEMM with the low-rank branch and bias fused:
  *   Y = bf16(deq(x_codes, x_scales) deq(w_codes, w_scales)^T + D L2 + bias),
  * float32 accumulation in tensor memory.  Inputs as produced by
- * svdq_quantize_act; Y device, M x N bf16.  Output tiles are 128 x 256 when
- * N % 256 == 0 and there are at least as many of them as SMs, else 128 x 128;
- * the environment variable SVDQ_GEMM_BN=128|256 overrides that choice.
+ * svdq_quantize_act; Y device, M x N bf16.  Single CTAs compute 128 x 256
+ * output tiles (N % 256 == 0 and at least one tile per SM) or 128 x 128 tiles
+ * (SVDQ_GEMM_BN=128|256 overrides); with SVDQ_GEMM_PAIR=1 and N % 256 == 0,
+ * CTA pairs compute 256 x 256 tiles with two-CTA MMAs instead.
  * ------------------------------------------------------------------------- */
 svdq_status svdq_gemm(const uint8_t* x_codes, const uint8_t* x_scales, const uint16_t* D, int M,
                       const svdq_weight* w, uint16_t* Y, void* stream);
@@ -240,6 +243,14 @@ svdq_status svdq_scales_to_native(const uint8_t* logical, int rows, int K, uint8
  * since the last clear.  *detail (optional) receives the raw word. */
 svdq_status svdq_get_device_status(void* stream, uint32_t* detail);
 svdq_status svdq_clear_device_status(void* stream);
+
+/* Failure-detection self-test: launch one bounded wait (the same kind every
+ * kernel of the library uses) on an mbarrier that nothing completes, with the
+ * given limit in nanoseconds (clamped to [1 us, 1 s]).  The wait gives up,
+ * records a timeout (kernel id 4, site 1) in the device status word and the
+ * kernel returns normally: the context stays usable.  Asynchronous on
+ * `stream`; read the result with svdq_get_device_status. */
+svdq_status svdq_selftest_wait_timeout(uint64_t limit_ns, void* stream);
 
 #ifdef __cplusplus
 }  /* extern "C" */

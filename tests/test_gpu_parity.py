@@ -212,10 +212,16 @@ def test_prepare_parity(N, K, r, with_bias):
 # S2 + S3: GEMM with fused low-rank branch and bias
 # ---------------------------------------------------------------------------
 
+@pytest.mark.parametrize("pair", [False, True], ids=["cta", "pair"])
 @pytest.mark.parametrize("M,K,N,r", [(256, 512, 512, 32), (1, 256, 128, 16), (129, 768, 384, 32),
-                                     (300, 1024, 256, 0), (64, 512, 1024, 64), (513, 256, 640, 8)])
-def test_gemm_parity(M, K, N, r):
-    """svdq_gemm on oracle-produced activation codes: isolates the tensor-core GEMM."""
+                                     (300, 1024, 256, 0), (64, 512, 1024, 64), (513, 256, 640, 8),
+                                     (700, 1280, 768, 48)])
+def test_gemm_parity(M, K, N, r, pair, monkeypatch):
+    """svdq_gemm on oracle-produced activation codes: isolates the tensor-core GEMM
+    (single-CTA 128-row tiles, or 256 x 256 tiles on CTA pairs)."""
+    if pair and N % 256:
+        pytest.skip("the CTA-pair kernel needs N % 256 == 0")
+    monkeypatch.setenv("SVDQ_GEMM_PAIR", "1" if pair else "0")
     t = torch()
     X, W, B, lam = _inputs(M, K, N, seed=3 * M + K + N + r)
     lin, exp = _prepare(W, lam, B, r)
@@ -237,10 +243,14 @@ def test_gemm_parity(M, K, N, r):
 # whole layer
 # ---------------------------------------------------------------------------
 
+@pytest.mark.parametrize("pair", [False, True], ids=["cta", "pair"])
 @pytest.mark.parametrize("M,K,N,r,with_bias", [(256, 512, 512, 32, True), (1, 256, 256, 32, True),
                                                (129, 1024, 384, 16, False), (777, 512, 1280, 64, True),
                                                (40, 768, 128, 0, False)])
-def test_forward_parity(M, K, N, r, with_bias):
+def test_forward_parity(M, K, N, r, with_bias, pair, monkeypatch):
+    if pair and N % 256:
+        pytest.skip("the CTA-pair kernel needs N % 256 == 0")
+    monkeypatch.setenv("SVDQ_GEMM_PAIR", "1" if pair else "0")
     t = torch()
     X, W, B, lam = _inputs(M, K, N, seed=11 * M + K + N + r)
     bias = B if with_bias else None

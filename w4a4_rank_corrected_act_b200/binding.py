@@ -62,6 +62,7 @@ SIGNATURES = {
     "svdq_scales_to_native": (_I, [_P, _I, _I, _P]),
     "svdq_get_device_status": (_I, [_P, ctypes.POINTER(ctypes.c_uint32)]),
     "svdq_clear_device_status": (_I, [_P]),
+    "svdq_selftest_wait_timeout": (_I, [ctypes.c_uint64, _P]),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -201,6 +202,10 @@ def svdq_get_device_status(stream: int = 0) -> int:
 
 def svdq_clear_device_status(stream: int = 0) -> None:
     _call("svdq_clear_device_status", stream or None)
+
+
+def svdq_selftest_wait_timeout(limit_ns: int, stream: int = 0) -> None:
+    _call("svdq_selftest_wait_timeout", int(limit_ns), stream or None)
 
 
 # --------------------------------------------------------------------------

@@ -13,20 +13,25 @@
 //   1. the low-rank term: R_PAD/16 bf16 MMAs (kind::f16, K = 16) of the D tile
 //      (128 x r) against the L2^T tile (BN x r) initialise the accumulator;
 //   2. K/64 block-scaled MMAs (kind::mxf4nvf4, K = 64, one UE4M3 scale per 16)
-//      accumulate the 4-bit product; scales are copied shared -> tensor memory
-//      with tcgen05.cp right before the MMAs that read them;
+//      accumulate the 4-bit product, reading the scales from tensor memory;
 //   3. the epilogue reads the accumulator with tcgen05.ld, adds the bias,
 //      rounds to bf16, stages 32 x 32 pieces in shared memory and stores Y
 //      with TMA.
 // Two accumulator buffers alternate between tiles so the epilogue of tile t
 // overlaps the MMAs of tile t+1.  With BN = 256 they cannot both fit next to
-// the scale columns (2 x 256 + 64 > 512), so buffer 1 starts at column 192 and
-// shares 64 columns with buffer 0; the epilogue reads those shared columns of a
+// the scale columns (2 x 256 + 96 > 512), so buffer 1 starts at column 160 and
+// shares 96 columns with buffer 0; the epilogue reads those shared columns of a
 // tile first and releases them before draining the rest.
-// Warp roles (256 threads): warp 0 issues TMA / bulk copies into a STAGES-deep
+// Scales reach tensor memory through registers, not through tcgen05.cp on the
+// MMA thread (each copy there costs the tensor pipe about as much as an MMA):
+// four scale warps read each stage's scale tiles from shared memory and write
+// them with tcgen05.st into one of two scale buffers, each lane quarter its own
+// replica of the layout the MMA reads; the MMA thread only waits for them.
+// Warp roles (384 threads): warp 0 issues TMA / bulk copies into a STAGES-deep
 // shared-memory ring, warp 1 issues the MMAs (one thread), warp 2 owns the
-// tensor-memory allocation, warps 4-7 run the epilogue (warp w reads lanes
-// 32*(w%4)..+31).  The grid is persistent (one CTA per SM, tiles strided).
+// tensor-memory allocation, warps 4-7 run the epilogue and warps 8-11 write
+// the scales (warp w accesses lanes 32*(w%4)..+31).  The grid is persistent
+// (one CTA per SM, tiles strided).
 #pragma once
 
 #include "nvfp4.cuh"
@@ -36,7 +41,7 @@ namespace svdq {
 
 constexpr int GEMM_BM = 128;
 constexpr int GEMM_BK = 256;                 // fp4 elements per stage = 128 bytes per row
-constexpr int GEMM_THREADS = 256;
+constexpr int GEMM_THREADS = 384;
 constexpr uint32_t GEMM_A_TILE = GEMM_BM * 128;   // 16 KB
 constexpr uint32_t GEMM_SFA_TILE = 4 * 512;       // 4 scale tiles (4 x 64 K) for 128 rows
 constexpr uint32_t GEMM_STAGE_OUT = 32 * 64;      // per epilogue warp: 32 rows x 32 bf16
@@ -56,16 +61,16 @@ struct GemmCfg {
   static constexpr uint32_t kStage = GEMM_A_TILE + kBTile + GEMM_SFA_TILE + kSFBTile;
   static constexpr int kStages = (BN == 256 ? 4 : 6);
   static constexpr uint32_t kTmemCols = 512;
-  // tensor-memory columns: scales in the top 64, accumulator buffers below
-  static constexpr uint32_t kSfaCol = 448;               // 4 k-blocks x 4 columns
-  static constexpr uint32_t kSfbCol = 464;               // 4 k-blocks x BN/32 columns
-  static constexpr uint32_t kAcc1Col = (BN == 256 ? 192 : 128);
-  static constexpr int kOverlapChunks = (BN == 256 ? (256 - 192) / 32 : 0);
+  // tensor-memory columns: two scale buffers in the top 96, accumulators below
+  static constexpr uint32_t kSfaCol0 = 416;              // + 16 j: 4 k-blocks x 4 columns
+  static constexpr uint32_t kSfbCol0 = 448;              // + 32 j: 4 k-blocks x BN/32 columns
+  static constexpr uint32_t kAcc1Col = (BN == 256 ? 160 : 128);
+  static constexpr int kOverlapChunks = (BN == 256 ? (256 - 160) / 32 : 0);
   static constexpr uint32_t kOutBytes = 4 * GEMM_STAGE_OUT;   // epilogue staging, 4 warps
-  static constexpr uint32_t kBarBytes = (2 * kStages + 4) * 8 + 16;
+  static constexpr uint32_t kBarBytes = (2 * kStages + 8) * 8 + 16;
   static constexpr uint32_t kSmemBytes = kStages * kStage + kOutBytes + kBarBytes + 1024;
-  static_assert(kSfbCol + 4 * (BN / 32) <= kTmemCols, "scale columns");
-  static_assert(kAcc1Col + BN <= kSfaCol, "accumulator buffer 1");
+  static_assert(kSfbCol0 + 32 + 4 * (BN / 32) <= kTmemCols, "scale columns");
+  static_assert(kAcc1Col + BN <= kSfaCol0, "accumulator buffer 1");
   static_assert(kStage % 1024 == 0, "stage alignment");
   static_assert(kSmemBytes <= 232448, "shared memory");
 };
@@ -102,8 +107,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* out_stage = smem + S * Cfg::kStage;
   uint64_t* bars = reinterpret_cast<uint64_t*>(out_stage + Cfg::kOutBytes);
-  // bars[0..S) full, [S..2S) empty, 2S/2S+1 tmem_full[2], 2S+2 tmem_free, 2S+3 drain
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 4);
+  // bars[0..S) full, [S..2S) empty, 2S/2S+1 tmem_full[2], 2S+2 tmem_free, 2S+3 drain,
+  // 2S+4/2S+5 sf_ready[2] (scale warps -> MMA), 2S+6/2S+7 sf_free[2] (MMA -> scale warps)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -119,6 +125,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   auto tmem_full = [&](int b) { return smem_u32(bars + 2 * S + b); };
   const uint32_t tmem_free = smem_u32(bars + 2 * S + 2);
   const uint32_t drain_bar = smem_u32(bars + 2 * S + 3);
+  auto sf_ready = [&](uint32_t b) { return smem_u32(bars + 2 * S + 4 + b); };
+  auto sf_free = [&](uint32_t b) { return smem_u32(bars + 2 * S + 6 + b); };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -129,6 +137,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     mbar_init(tmem_full(1), 1);
     mbar_init(tmem_free, 128);
     mbar_init(drain_bar, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(sf_ready(b), 128);
+      mbar_init(sf_free(b), 1);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -203,6 +215,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       bool ok = true;
       bool any_issued = false;
       int local = 0;   // tiles issued by this CTA
+      uint32_t n = 0;  // k-blocks issued (selects the scale buffer)
       for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x, ++local) {
         const int buf = local & 1;
         const uint32_t acc = tmem_base + (buf ? Cfg::kAcc1Col : 0u);
@@ -232,29 +245,21 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         }
         for (int kb = 0; kb < kb_per_tile; ++kb) {
           if (!mbar_wait(full_bar(stage), phase, abort_flag, KID_GEMM, 6)) { ok = false; break; }
+          const uint32_t sb = n & 1u;
+          if (!mbar_wait(sf_ready(sb), (n >> 1) & 1u, abort_flag, KID_GEMM, 9)) { ok = false; break; }
           tc_fence_after();
-          // scale factors: shared -> tensor memory (32 rows x 16 B per copy); the
-          // region is reused by every stage (tcgen05 ops of a thread run in order)
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            tc_cp_32x128b_warpx4(tmem_base + Cfg::kSfaCol + 4 * i,
-                                 make_smem_desc(stage_sfa(stage) + i * 512, LAYOUT_NONE, 128, 0));
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int g = 0; g < BN / 128; ++g)
-              tc_cp_32x128b_warpx4(
-                  tmem_base + Cfg::kSfbCol + i * (BN / 32) + 4 * g,
-                  make_smem_desc(stage_sfb(stage) + (g * 4 + i) * 512, LAYOUT_NONE, 128, 0));
+          const uint32_t sfa = tmem_base + Cfg::kSfaCol0 + 16 * sb;
+          const uint32_t sfb = tmem_base + Cfg::kSfbCol0 + 32 * sb;
           const uint64_t ad = make_smem_desc(stage_a(stage), LAYOUT_SW128, 1024, 0);
           const uint64_t bd = make_smem_desc(stage_b(stage), LAYOUT_SW128, 1024, 0);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            tc_mma_nvfp4(acc, ad + 2 * i, bd + 2 * i, idf, tmem_base + Cfg::kSfaCol + 4 * i,
-                         tmem_base + Cfg::kSfbCol + i * (BN / 32), accumulate);
+            tc_mma_nvfp4(acc, ad + 2 * i, bd + 2 * i, idf, sfa + 4 * i, sfb + i * (BN / 32), accumulate);
             accumulate = 1;
           }
           tc_commit(empty_bar(stage));
+          tc_commit(sf_free(sb));
+          ++n;
           any_issued = true;
           if (++stage == S) { stage = 0; phase ^= 1; }
         }
@@ -267,7 +272,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         mbar_wait_drain(drain_bar, 0);
       }
     }
-  } else if (warp >= 4) {
+  } else if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
     uint8_t* stg = out_stage + q * GEMM_STAGE_OUT;
@@ -333,6 +338,65 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
     if (lane == 0) bulk_wait_group_all();
     __syncwarp();
+  } else if (warp >= 8) {
+    // ------------------------------------------------------------ scale warps
+    // Each lane quarter gets its replica of the layout the MMA reads: for
+    // k-block i of a stage, 4 columns of A scales and BN/32 columns of B
+    // scales, column (4 i + g) / (BN/32 i + g) of lane 32 q + l holding the 4
+    // scales of row 32 g + l -- exactly the 16 bytes at offset 16 l of the
+    // 512-byte scale tile in shared memory.
+    const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    int stage = 0;
+    uint32_t phase = 0, n = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+      if (R_PAD > 0) {
+        if (++stage == S) { stage = 0; phase ^= 1; }
+      }
+      for (int kb = 0; kb < kb_per_tile; ++kb) {
+        if (!mbar_wait(full_bar(stage), phase, abort_flag, KID_GEMM, 20)) { ok = false; break; }
+        const uint32_t sb = n & 1u;
+        if (n >= 2 && !mbar_wait(sf_free(sb), ((n >> 1) - 1) & 1u, abort_flag, KID_GEMM, 21)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint8_t* sa = smem + (stage_sfa(stage) - smem_base) + lane * 16;
+        const uint8_t* sbp = smem + (stage_sfb(stage) - smem_base) + lane * 16;
+        uint32_t va[16];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint4 x = *reinterpret_cast<const uint4*>(sa + i * 512);
+          va[4 * i] = x.x; va[4 * i + 1] = x.y; va[4 * i + 2] = x.z; va[4 * i + 3] = x.w;
+        }
+        tmem_st_32x32b_x16(tmem_base + lane_addr + Cfg::kSfaCol0 + 16 * sb, va);
+        if (BN == 256) {
+          uint32_t vb[32];
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int g = 0; g < 2; ++g) {
+              const uint4 x = *reinterpret_cast<const uint4*>(sbp + (g * 4 + i) * 512);
+              vb[8 * i + 4 * g] = x.x; vb[8 * i + 4 * g + 1] = x.y;
+              vb[8 * i + 4 * g + 2] = x.z; vb[8 * i + 4 * g + 3] = x.w;
+            }
+          tmem_st_32x32b_x32(tmem_base + lane_addr + Cfg::kSfbCol0 + 32 * sb, vb);
+        } else {
+          uint32_t vb[16];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint4 x = *reinterpret_cast<const uint4*>(sbp + i * 512);
+            vb[4 * i] = x.x; vb[4 * i + 1] = x.y; vb[4 * i + 2] = x.z; vb[4 * i + 3] = x.w;
+          }
+          tmem_st_32x32b_x16(tmem_base + lane_addr + Cfg::kSfbCol0 + 32 * sb, vb);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(sf_ready(sb));
+        ++n;
+        if (++stage == S) { stage = 0; phase ^= 1; }
+      }
+    }
   }
 
   tc_fence_before();

@@ -25,6 +25,7 @@
 #include "svdq.h"
 #include "act_quant.cuh"
 #include "fp4_gemm.cuh"
+#include "fp4_gemm_pair.cuh"
 #include "prepare.cuh"
 
 using namespace svdq;
@@ -214,8 +215,79 @@ svdq_status quantize_act_impl(const uint16_t* X, int M, const svdq_weight* w, ui
   }
 }
 
+template <int R_PAD>
+svdq_status launch_gemm_pair(const CUtensorMap* maps, const GemmPairParams& p, int num_pairs,
+                             cudaStream_t st) {
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(fp4_gemm_pair_kernel<R_PAD>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, GemmPairCfg::kSmemBytes);
+  });
+  if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(gemm pair)");
+  fp4_gemm_pair_kernel<R_PAD><<<2 * num_pairs, GP_THREADS, GemmPairCfg::kSmemBytes, st>>>(
+      maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6], p);
+  SVDQ_CHECK_LAUNCH("fp4_gemm_pair_kernel");
+  return SVDQ_OK;
+}
+
+// 256 x 256 tiles on CTA pairs (see fp4_gemm_pair.cuh).
+svdq_status gemm_pair_impl(const uint8_t* x_codes, const uint8_t* x_scales, const uint16_t* D, int M,
+                           const svdq_weight* w, uint16_t* Y, cudaStream_t st) {
+  const int N = w->N, K = w->K, r = w->r, rp = r_pad_of(r);
+  CUtensorMap maps[7] = {};   // a, b, sfa, sfb, d, l2, y
+  svdq_status s = make_tmap(&maps[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, x_codes, K / 2, M, K / 2, 128, 128,
+                            CU_TENSOR_MAP_SWIZZLE_128B);
+  if (s != SVDQ_OK) return s;
+  s = make_tmap(&maps[1], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->w_codes, K / 2, N, K / 2, 128, 128,
+                CU_TENSOR_MAP_SWIZZLE_128B);
+  if (s != SVDQ_OK) return s;
+  // scale tiles of one 128-row block form a row of K * 8 bytes; a 256-wide K
+  // stage is 2 KB of it (256 elements of 8 bytes)
+  s = make_tmap(&maps[2], CU_TENSOR_MAP_DATA_TYPE_UINT64, x_scales, K, m_pad_of(M) / 128,
+                static_cast<uint64_t>(K) * 8, 256, 1, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (s != SVDQ_OK) return s;
+  s = make_tmap(&maps[3], CU_TENSOR_MAP_DATA_TYPE_UINT64, w->w_scales, K, N / 128,
+                static_cast<uint64_t>(K) * 8, 256, 2, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (s != SVDQ_OK) return s;
+  if (r > 0) {
+    s = make_tmap(&maps[4], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, D, r, M, static_cast<uint64_t>(r) * 2, rp,
+                  128, lr_swizzle(rp));
+    if (s != SVDQ_OK) return s;
+    s = make_tmap(&maps[5], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->L2t, r, N,
+                  static_cast<uint64_t>(r) * 2, rp, 128, lr_swizzle(rp));
+    if (s != SVDQ_OK) return s;
+  }
+  s = make_tmap(&maps[6], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, N, M, static_cast<uint64_t>(N) * 2, 32, 32,
+                CU_TENSOR_MAP_SWIZZLE_64B);
+  if (s != SVDQ_OK) return s;
+  GemmPairParams p;
+  p.bias = w->has_bias ? w->bias : nullptr;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.r = r;
+  p.m_tiles = (M + GP_BM - 1) / GP_BM;
+  p.n_tiles = N / GP_BN;
+  p.num_tiles = p.m_tiles * p.n_tiles;
+  p.kblocks = K / GEMM_BK;
+  const int num_pairs = std::max(1, std::min(p.num_tiles, num_sms() / 2));
+  switch (rp) {
+    case 0: return launch_gemm_pair<0>(maps, p, num_pairs, st);
+    case 16: return launch_gemm_pair<16>(maps, p, num_pairs, st);
+    case 32: return launch_gemm_pair<32>(maps, p, num_pairs, st);
+    default: return launch_gemm_pair<64>(maps, p, num_pairs, st);
+  }
+}
+
 svdq_status gemm_impl(const uint8_t* x_codes, const uint8_t* x_scales, const uint16_t* D, int M,
                       const svdq_weight* w, uint16_t* Y, cudaStream_t st) {
+  {
+    // the CTA-pair kernel (256 x 256 tiles) is used on request (SVDQ_GEMM_PAIR=1)
+    bool pair = false;
+    if (const char* e = std::getenv("SVDQ_GEMM_PAIR")) pair = (std::atoi(e) != 0) && (w->N % 256 == 0);
+    if (pair) return gemm_pair_impl(x_codes, x_scales, D, M, w, Y, st);
+  }
   const int N = w->N, K = w->K, r = w->r, rp = r_pad_of(r);
   const int m_tiles = (M + GEMM_BM - 1) / GEMM_BM;
   // 256-wide tiles when N allows it and there are enough of them to fill the GPU
@@ -361,6 +433,24 @@ void to_logical(const uint8_t* native, int rows, int K, uint8_t* logical) {
   for (int i = 0; i < rows; ++i)
     for (int j = 0; j < kb; ++j)
       logical[static_cast<size_t>(i) * kb + j] = native[sf_offset(i, j, K)];
+}
+
+// One bounded wait on an mbarrier that nothing arrives on: the same wait the
+// layer's kernels use, made to run out, so the timeout path (status word,
+// clean return) can be tested without faulting or hanging the GPU.
+__global__ void selftest_wait_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(smem_u32(&bar), 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0)
+    mbar_wait(smem_u32(&bar), 0, reinterpret_cast<volatile int*>(&abort_flag), KID_SELFTEST, 1,
+              limit_ns);
+  __syncthreads();
 }
 
 // --------------------------------------------------------------------------
@@ -675,6 +765,14 @@ svdq_status svdq_get_device_status(void* stream, uint32_t* detail) {
   SVDQ_CUDA(cudaMemcpyFromSymbol(&v, g_device_status, sizeof(v)));
   if (detail) *detail = v;
   return v ? SVDQ_ERR_TIMEOUT : SVDQ_OK;
+}
+
+svdq_status svdq_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
+  const unsigned long long lim =
+      std::min<unsigned long long>(std::max<unsigned long long>(limit_ns, 1000ull), 1000000000ull);
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(lim);
+  SVDQ_CHECK_LAUNCH("selftest_wait_kernel");
+  return SVDQ_OK;
 }
 
 svdq_status svdq_clear_device_status(void* stream) {
