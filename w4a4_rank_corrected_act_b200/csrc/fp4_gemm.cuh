@@ -44,7 +44,8 @@ constexpr int GEMM_BK = 256;                 // fp4 elements per stage = 128 byt
 constexpr int GEMM_THREADS = 384;
 constexpr uint32_t GEMM_A_TILE = GEMM_BM * 128;   // 16 KB
 constexpr uint32_t GEMM_SFA_TILE = 4 * 512;       // 4 scale tiles (4 x 64 K) for 128 rows
-constexpr uint32_t GEMM_STAGE_OUT = 32 * 64;      // per epilogue warp: 32 rows x 32 bf16
+constexpr uint32_t GEMM_OUT_PIECE = 32 * 32;      // 32 rows x 16 bf16, 32-byte swizzle
+constexpr uint32_t GEMM_STAGE_OUT = 2 * GEMM_OUT_PIECE;   // per epilogue warp: two pieces
 
 struct GemmParams {
   const uint8_t* x_scales;
@@ -91,6 +92,99 @@ __host__ __device__ constexpr uint32_t idesc_nvfp4(int M, int N) {
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// Bias of columns n0 .. n0 + BN - 1, 16 bytes per lane (lane l holds columns
+// n0 + 8 l .. n0 + 8 l + 7); loaded before the accumulator is ready so that its
+// latency is hidden, and handed out with shuffles.
+template <int BN>
+__device__ __forceinline__ uint4 load_tile_bias(const uint16_t* bias, int n0, int lane) {
+  uint4 b = make_uint4(0u, 0u, 0u, 0u);
+  if (bias != nullptr && lane < BN / 8) b = __ldg(reinterpret_cast<const uint4*>(bias + n0) + lane);
+  return b;
+}
+
+// One 32-row x 16-column piece of the output for the warp owning the rows
+// row0 .. row0 + 31 (lane = row): accumulator bits `v` plus bias, rounded to
+// bf16, staged in one of two 32-byte-swizzled 1 KB buffers and stored with
+// TMA.  A store may still be reading the other buffer.
+__device__ __forceinline__ void store_piece(const uint32_t (&v)[16], int slot, int c, int lane,
+                                            bool has_bias, uint4 bias, int n0, int row0,
+                                            const CUtensorMap* tm_y, uint8_t* stg, uint32_t stg_u) {
+  float f[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) f[j] = __uint_as_float(v[j]);
+  if (has_bias) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int src = 2 * c + u;
+      const uint32_t bw[4] = {__shfl_sync(0xffffffffu, bias.x, src), __shfl_sync(0xffffffffu, bias.y, src),
+                              __shfl_sync(0xffffffffu, bias.z, src), __shfl_sync(0xffffffffu, bias.w, src)};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        f[u * 8 + 2 * h] += bf16_bits_to_f32(bw[h] & 0xFFFFu);
+        f[u * 8 + 2 * h + 1] += bf16_bits_to_f32(bw[h] >> 16);
+      }
+    }
+  }
+  // the store issued two pieces ago must have finished reading this buffer
+  if (lane == 0) bulk_wait_group_read<1>();
+  __syncwarp();
+  uint8_t* buf = stg + slot * GEMM_OUT_PIECE;
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    uint4 o;
+    o.x = pack_bf16x2(f[u * 8 + 0], f[u * 8 + 1]);
+    o.y = pack_bf16x2(f[u * 8 + 2], f[u * 8 + 3]);
+    o.z = pack_bf16x2(f[u * 8 + 4], f[u * 8 + 5]);
+    o.w = pack_bf16x2(f[u * 8 + 6], f[u * 8 + 7]);
+    *reinterpret_cast<uint4*>(buf + swz(lane * 32 + u * 16, 1)) = o;
+  }
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(tm_y, stg_u + slot * GEMM_OUT_PIECE, n0 + c * 16, row0);
+    bulk_commit_group();
+  }
+}
+
+// Epilogue of one 128 x BN tile for the warp owning tensor-memory lanes
+// 32 q .. 32 q + 31 (= tile rows), in 16-column pieces taken in `order`.  The
+// first KOV pieces are the columns the next tile's accumulator shares: they
+// are read together, `release` runs after that single wait, and only then are
+// they converted and stored.  The remaining pieces are read one ahead of the
+// one being stored.  `bias` is the tile's bias from load_tile_bias.
+template <int BN, int KOV, typename Order, typename Release>
+__device__ __forceinline__ void epilogue_tile(uint32_t acc, uint32_t lane_addr, int lane,
+                                              bool has_bias, uint4 bias, int n0, int row0,
+                                              const CUtensorMap* tm_y, uint8_t* stg, uint32_t stg_u,
+                                              Order order, Release release) {
+  constexpr int kPieces = BN / 16;
+  static_assert(KOV % 2 == 0 && KOV < kPieces, "shared pieces: an even count below the tile's");
+  uint32_t v[2][16];
+  if constexpr (KOV > 0) {
+    uint32_t ov[KOV][16];
+#pragma unroll
+    for (int j = 0; j < KOV; ++j) tmem_ld_32x32b_x16(acc + lane_addr + order(j) * 16, ov[j]);
+    tmem_ld_wait();
+    tc_fence_before();
+    release();
+    tmem_ld_32x32b_x16(acc + lane_addr + order(KOV) * 16, v[0]);
+#pragma unroll
+    for (int j = 0; j < KOV; ++j)
+      store_piece(ov[j], j & 1, order(j), lane, has_bias, bias, n0, row0, tm_y, stg, stg_u);
+  } else {
+    tc_fence_before();
+    release();
+    tmem_ld_32x32b_x16(acc + lane_addr + order(0) * 16, v[0]);
+  }
+  tmem_ld_wait();
+#pragma unroll 2
+  for (int i = KOV; i < kPieces; ++i) {
+    if (i + 1 < kPieces) tmem_ld_32x32b_x16(acc + lane_addr + order(i + 1) * 16, v[(i + 1) & 1]);
+    store_piece(v[i & 1], i & 1, order(i), lane, has_bias, bias, n0, row0, tm_y, stg, stg_u);
+    tmem_ld_wait();
+  }
+}
+
 template <int BN, int R_PAD>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     fp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
@@ -100,7 +194,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   constexpr int S = Cfg::kStages;
   constexpr uint32_t kLRLayout = (R_PAD == 64 ? LAYOUT_SW128 : R_PAD == 32 ? LAYOUT_SW64 : LAYOUT_SW32);
   constexpr uint32_t kLRSbo = 8 * R_PAD * 2;
-  constexpr int kChunks = BN / 32;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -284,57 +377,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       const int m0 = mb * GEMM_BM, n0 = nb * BN;
       const int buf = local & 1;
       const uint32_t acc = tmem_base + (buf ? Cfg::kAcc1Col : 0u);
+      const uint4 tile_bias = load_tile_bias<BN>(p.bias, n0, lane);
       if (!mbar_wait(tmem_full(buf), static_cast<uint32_t>(local >> 1) & 1u, abort_flag, KID_GEMM, 8))
         break;
       tc_fence_after();
-#pragma unroll 1
-      for (int i = 0; i < kChunks; ++i) {
-        // buffer 0 shares its top chunks with buffer 1, buffer 1 its bottom
-        // chunks with buffer 0: those come first, then the columns are released
-        const int c = buf ? i : (i + kChunks - Cfg::kOverlapChunks) % kChunks;
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(acc + lane_addr + c * 32, v);
-        tmem_ld_wait();
-        if (i + 1 == Cfg::kOverlapChunks || (Cfg::kOverlapChunks == 0 && i == 0)) {
-          tc_fence_before();
-          mbar_arrive(tmem_free);
-        }
-        float f[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[j]);
-        if (p.bias != nullptr) {
-          const uint4* bp = reinterpret_cast<const uint4*>(p.bias + n0 + c * 32);
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const uint4 b = __ldg(bp + u);
-            const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-              f[u * 8 + 2 * h] += bf16_bits_to_f32(bw[h] & 0xFFFFu);
-              f[u * 8 + 2 * h + 1] += bf16_bits_to_f32(bw[h] >> 16);
-            }
-          }
-        }
-        // the previous store of this warp must have finished reading the staging
-        if (lane == 0) bulk_wait_group_read<0>();
-        __syncwarp();
-        // row `lane` of the 32 x 32 piece, 64-byte swizzled (the TMA store's layout)
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          uint4 o;
-          o.x = pack_bf16x2(f[u * 8 + 0], f[u * 8 + 1]);
-          o.y = pack_bf16x2(f[u * 8 + 2], f[u * 8 + 3]);
-          o.z = pack_bf16x2(f[u * 8 + 4], f[u * 8 + 5]);
-          o.w = pack_bf16x2(f[u * 8 + 6], f[u * 8 + 7]);
-          *reinterpret_cast<uint4*>(stg + swz(lane * 64 + u * 16, 2)) = o;
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_2d(&tm_y, stg_u, n0 + c * 32, m0 + q * 32);
-          bulk_commit_group();
-        }
-      }
+      // buffer 0 shares its top columns with buffer 1, buffer 1 its bottom
+      // columns with buffer 0: those pieces come first
+      constexpr int kPieces = BN / 16, kOv = 2 * Cfg::kOverlapChunks;
+      epilogue_tile<BN, kOv>(
+          acc, lane_addr, lane, p.bias != nullptr, tile_bias, n0, m0 + q * 32, &tm_y, stg, stg_u,
+          [&](int i) { return buf ? i : (i + kPieces - kOv) % kPieces; },
+          [&]() { mbar_arrive(tmem_free); });
     }
     if (lane == 0) bulk_wait_group_all();
     __syncwarp();

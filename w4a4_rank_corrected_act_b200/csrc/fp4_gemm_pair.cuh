@@ -14,10 +14,12 @@
 // every byte of B's codes is loaded once per pair instead of once per CTA (38 KB
 // of operands per CTA per 256-wide K stage instead of 54 KB).  B's scales are
 // needed whole in each CTA's tensor memory (each CTA computes all 256 columns
-// of its rows), so both CTAs load the scale rows of the full 256-row B tile.  The leader (rank
-// 0) issues the MMAs and the scale copies; every TMA load of both CTAs
-// completes on the leader's stage barrier; MMA completion is signalled to the
-// barriers of both CTAs.  Each CTA's tensor memory holds its 128 rows of the
+// of its rows), so both CTAs load the scale rows of the full 256-row B tile.
+// The leader (rank 0) issues the MMAs; the code tiles of both CTAs complete on
+// the leader's stage barrier, each CTA's scale tiles on its own, and each CTA's
+// scale warps write its tensor-memory scale buffers with tcgen05.st (as in the
+// single-CTA kernel) and report to the leader; MMA completion is signalled to
+// the barriers of both CTAs.  Each CTA's tensor memory holds its 128 rows of the
 // fp32 accumulator (two alternating 256-column buffers sharing 64 columns, as
 // in the single-CTA kernel) and its scale columns.  Each CTA's epilogue stores
 // its own 128 rows and releases the shared columns to the leader.
@@ -29,7 +31,7 @@
 
 namespace svdq {
 
-constexpr int GP_THREADS = 256;
+constexpr int GP_THREADS = 384;
 constexpr int GP_BM = 256;                 // tile rows per pair (128 per CTA)
 constexpr int GP_BN = 256;                 // tile columns per pair (128 B rows per CTA)
 constexpr uint32_t GP_A_TILE = 128 * 128;  // 16 KB per CTA and stage
@@ -41,12 +43,12 @@ struct GemmPairCfg {
   static constexpr uint32_t kStage = GP_A_TILE + GP_B_TILE + GP_SF_TILE + GP_SFB_TILE;   // 38 KB
   static constexpr int kStages = 5;
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kSfaCol = 448;    // 4 k-blocks x 4 columns
-  static constexpr uint32_t kSfbCol = 464;    // 4 k-blocks x 8 columns (all 256 B rows)
-  static constexpr uint32_t kAcc1Col = 192;
-  static constexpr int kOverlapChunks = 2;
+  static constexpr uint32_t kSfaCol0 = 416;   // + 16 j: 4 k-blocks x 4 columns
+  static constexpr uint32_t kSfbCol0 = 448;   // + 32 j: 4 k-blocks x 8 columns (all 256 B rows)
+  static constexpr uint32_t kAcc1Col = 160;
+  static constexpr int kOverlapChunks = 3;
   static constexpr uint32_t kOutBytes = 4 * GEMM_STAGE_OUT;
-  static constexpr uint32_t kBarBytes = (2 * kStages + 4) * 8 + 16;
+  static constexpr uint32_t kBarBytes = (3 * kStages + 8) * 8 + 16;
   static constexpr uint32_t kSmemBytes = kStages * kStage + kOutBytes + kBarBytes + 1024;
   static_assert(kSmemBytes <= 232448, "shared memory");
   static_assert(kStage % 1024 == 0, "stage alignment");
@@ -68,16 +70,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GP_THREADS, 1)
   constexpr int S = Cfg::kStages;
   constexpr uint32_t kLRLayout = (R_PAD == 64 ? LAYOUT_SW128 : R_PAD == 32 ? LAYOUT_SW64 : LAYOUT_SW32);
   constexpr uint32_t kLRSbo = 8 * R_PAD * 2;
-  constexpr int kChunks = GP_BN / 32;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* out_stage = smem + S * Cfg::kStage;
   uint64_t* bars = reinterpret_cast<uint64_t*>(out_stage + Cfg::kOutBytes);
-  // bars[0..S) full (the leader's count both CTAs), [S..2S) empty,
-  // 2S/2S+1 tmem_full[2], 2S+2 tmem_free (the leader's counts both epilogues), 2S+3 drain
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 4);
+  // bars[0..S) full (code tiles; the leader's counts both CTAs), [S..2S) empty,
+  // 2S/2S+1 tmem_full[2], 2S+2 tmem_free (the leader's counts both epilogues), 2S+3 drain,
+  // 2S+4/2S+5 sf_ready[2] (the leader's counts both CTAs' scale warps),
+  // 2S+6/2S+7 sf_free[2], [2S+8..3S+8) sf_full (this CTA's scale tiles)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * S + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -95,6 +98,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GP_THREADS, 1)
   auto tmem_full = [&](int b) { return smem_u32(bars + 2 * S + b); };
   const uint32_t tmem_free = smem_u32(bars + 2 * S + 2);
   const uint32_t drain_bar = smem_u32(bars + 2 * S + 3);
+  auto sf_ready = [&](uint32_t b) { return smem_u32(bars + 2 * S + 4 + b); };
+  auto sf_free = [&](uint32_t b) { return smem_u32(bars + 2 * S + 6 + b); };
+  auto sf_full = [&](int st) { return smem_u32(bars + 2 * S + 8 + st); };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -105,6 +111,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GP_THREADS, 1)
     mbar_init(tmem_full(1), 1);
     mbar_init(tmem_free, 2 * 128);    // both CTAs' epilogue threads
     mbar_init(drain_bar, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(sf_ready(b), 2 * 128);  // both CTAs' scale warps
+      mbar_init(sf_free(b), 1);         // one multicast MMA commit
+    }
+    for (int st = 0; st < S; ++st) mbar_init(sf_full(st), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -137,7 +148,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GP_THREADS, 1)
       uint32_t phase = 0;
       int8_t fill_parity[S];
       for (int s = 0; s < S; ++s) fill_parity[s] = -1;
-      const uint32_t tx_main = 2 * Cfg::kStage;                  // both CTAs' bytes
+      const uint32_t tx_main = 2 * (GP_A_TILE + GP_B_TILE);      // both CTAs' code tiles
       const uint32_t tx_lr = 2 * (128 + 128) * R_PAD * 2;
       // arm (leader) or announce (peer) this CTA's loads for a stage
       auto post = [&](int s, uint32_t tx) {
@@ -154,6 +165,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GP_THREADS, 1)
           tma_load_2d_pair(stage_a(stage), &tm_d, lb, 0, m0);
           tma_load_2d_pair(stage_b(stage), &tm_l2, lb, 0, n0);
           post(stage, tx_lr);
+          mbar_arrive(sf_full(stage));   // keeps sf_full's phases in step with the ring
           fill_parity[stage] = static_cast<int8_t>(phase);
           if (++stage == S) { stage = 0; phase ^= 1; }
         }
@@ -162,16 +174,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GP_THREADS, 1)
           const uint32_t lb = leader_bar(full_bar(stage));
           tma_load_2d_pair(stage_a(stage), &tm_a, lb, kb * 128, m0);
           tma_load_2d_pair(stage_b(stage), &tm_b, lb, kb * 128, n0);
-          tma_load_2d_pair(stage_sfa(stage), &tm_sfa, lb, kb * 256, m0 / 128);
-          tma_load_2d_pair(stage_sfb(stage), &tm_sfb, lb, kb * 256, (n0 - 128 * rank) / 128);
           post(stage, tx_main);
+          mbar_arrive_expect_tx(sf_full(stage), GP_SF_TILE + GP_SFB_TILE);
+          tma_load_2d(stage_sfa(stage), &tm_sfa, sf_full(stage), kb * 256, m0 / 128);
+          tma_load_2d(stage_sfb(stage), &tm_sfb, sf_full(stage), kb * 256, (n0 - 128 * rank) / 128);
           fill_parity[stage] = static_cast<int8_t>(phase);
           if (++stage == S) { stage = 0; phase ^= 1; }
         }
       }
-      if (*abort_flag && leader) {
+      if (*abort_flag) {
         for (int s = 0; s < S; ++s)
-          if (fill_parity[s] >= 0) mbar_wait_drain(full_bar(s), static_cast<uint32_t>(fill_parity[s]));
+          if (fill_parity[s] >= 0) {
+            if (leader) mbar_wait_drain(full_bar(s), static_cast<uint32_t>(fill_parity[s]));
+            mbar_wait_drain(sf_full(s), static_cast<uint32_t>(fill_parity[s]));
+          }
       }
     }
   } else if (warp == 1) {
@@ -184,6 +200,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GP_THREADS, 1)
       bool ok = true;
       bool any_issued = false;
       int local = 0;
+      uint32_t n = 0;
       for (int t = pair; t < p.num_tiles && ok; t += num_pairs, ++local) {
         const int buf = local & 1;
         const uint32_t acc = tmem_base + (buf ? Cfg::kAcc1Col : 0u);
@@ -211,26 +228,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GP_THREADS, 1)
         }
         for (int kb = 0; kb < kb_per_tile; ++kb) {
           if (!mbar_wait(full_bar(stage), phase, abort_flag, KID_GEMM, 16)) { ok = false; break; }
+          const uint32_t sb = n & 1u;
+          if (!mbar_wait(sf_ready(sb), (n >> 1) & 1u, abort_flag, KID_GEMM, 17)) { ok = false; break; }
           tc_fence_after();
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            tc_cp_pair_32x128b_warpx4(tmem_base + Cfg::kSfaCol + 4 * i,
-                                      make_smem_desc(stage_sfa(stage) + i * 512, LAYOUT_NONE, 128, 0));
-#pragma unroll
-            for (int g = 0; g < 2; ++g)
-              tc_cp_pair_32x128b_warpx4(
-                  tmem_base + Cfg::kSfbCol + 8 * i + 4 * g,
-                  make_smem_desc(stage_sfb(stage) + g * GP_SF_TILE + i * 512, LAYOUT_NONE, 128, 0));
-          }
+          const uint32_t sfa = tmem_base + Cfg::kSfaCol0 + 16 * sb;
+          const uint32_t sfb = tmem_base + Cfg::kSfbCol0 + 32 * sb;
           const uint64_t ad = make_smem_desc(stage_a(stage), LAYOUT_SW128, 1024, 0);
           const uint64_t bd = make_smem_desc(stage_b(stage), LAYOUT_SW128, 1024, 0);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            tc_mma_nvfp4_pair(acc, ad + 2 * i, bd + 2 * i, idf, tmem_base + Cfg::kSfaCol + 4 * i,
-                              tmem_base + Cfg::kSfbCol + 8 * i, accumulate);
+            tc_mma_nvfp4_pair(acc, ad + 2 * i, bd + 2 * i, idf, sfa + 4 * i, sfb + 8 * i, accumulate);
             accumulate = 1;
           }
           tc_commit_pair(empty_bar(stage));
+          tc_commit_pair(sf_free(sb));
+          ++n;
           any_issued = true;
           if (++stage == S) { stage = 0; phase ^= 1; }
         }
@@ -242,7 +254,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GP_THREADS, 1)
         mbar_wait_drain(drain_bar, 0);
       }
     }
-  } else if (warp >= 4) {
+  } else if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int q = warp & 3;
     uint8_t* stg = out_stage + q * GEMM_STAGE_OUT;
@@ -255,56 +267,65 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GP_THREADS, 1)
       const int m0 = mb * GP_BM + 128 * rank, n0 = nb * GP_BN;
       const int buf = local & 1;
       const uint32_t acc = tmem_base + (buf ? Cfg::kAcc1Col : 0u);
+      const uint4 tile_bias = load_tile_bias<GP_BN>(p.bias, n0, lane);
       if (!mbar_wait(tmem_full(buf), static_cast<uint32_t>(local >> 1) & 1u, abort_flag, KID_GEMM, 18))
         break;
       tc_fence_after();
-#pragma unroll 1
-      for (int i = 0; i < kChunks; ++i) {
-        const int c = buf ? i : (i + kChunks - Cfg::kOverlapChunks) % kChunks;
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(acc + lane_addr + c * 32, v);
-        tmem_ld_wait();
-        if (i + 1 == Cfg::kOverlapChunks) {
-          tc_fence_before();
-          mbar_arrive_cluster(leader_free);
-        }
-        float f[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[j]);
-        if (p.bias != nullptr) {
-          const uint4* bp = reinterpret_cast<const uint4*>(p.bias + n0 + c * 32);
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const uint4 b = __ldg(bp + u);
-            const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-              f[u * 8 + 2 * h] += bf16_bits_to_f32(bw[h] & 0xFFFFu);
-              f[u * 8 + 2 * h + 1] += bf16_bits_to_f32(bw[h] >> 16);
-            }
-          }
-        }
-        if (lane == 0) bulk_wait_group_read<0>();
-        __syncwarp();
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          uint4 o;
-          o.x = pack_bf16x2(f[u * 8 + 0], f[u * 8 + 1]);
-          o.y = pack_bf16x2(f[u * 8 + 2], f[u * 8 + 3]);
-          o.z = pack_bf16x2(f[u * 8 + 4], f[u * 8 + 5]);
-          o.w = pack_bf16x2(f[u * 8 + 6], f[u * 8 + 7]);
-          *reinterpret_cast<uint4*>(stg + swz(lane * 64 + u * 16, 2)) = o;
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_2d(&tm_y, stg_u, n0 + c * 32, m0 + q * 32);
-          bulk_commit_group();
-        }
-      }
+      constexpr int kPieces = GP_BN / 16, kOv = 2 * Cfg::kOverlapChunks;
+      epilogue_tile<GP_BN, kOv>(
+          acc, lane_addr, lane, p.bias != nullptr, tile_bias, n0, m0 + q * 32, &tm_y, stg, stg_u,
+          [&](int i) { return buf ? i : (i + kPieces - kOv) % kPieces; },
+          [&]() { mbar_arrive_cluster(leader_free); });
     }
     if (lane == 0) bulk_wait_group_all();
     __syncwarp();
+  } else if (warp >= 8) {
+    // ------------------------------------------------------------ scale warps (both CTAs)
+    // this CTA's tensor memory: A scales of its 128 rows, B scales of all 256
+    // tile columns, each lane quarter its replica (see fp4_gemm.cuh)
+    const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t leader_ready0 = mapa_shared(sf_ready(0), 0);
+    int stage = 0;
+    uint32_t phase = 0, n = 0;
+    bool ok = true;
+    for (int t = pair; t < p.num_tiles && ok; t += num_pairs) {
+      if (R_PAD > 0) {
+        if (++stage == S) { stage = 0; phase ^= 1; }
+      }
+      for (int kb = 0; kb < kb_per_tile; ++kb) {
+        if (!mbar_wait(sf_full(stage), phase, abort_flag, KID_GEMM, 20)) { ok = false; break; }
+        const uint32_t sb = n & 1u;
+        if (n >= 2 && !mbar_wait(sf_free(sb), ((n >> 1) - 1) & 1u, abort_flag, KID_GEMM, 21)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint8_t* sa = smem + (stage_sfa(stage) - smem_base) + lane * 16;
+        const uint8_t* sbp = smem + (stage_sfb(stage) - smem_base) + lane * 16;
+        uint32_t va[16];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint4 x = *reinterpret_cast<const uint4*>(sa + i * 512);
+          va[4 * i] = x.x; va[4 * i + 1] = x.y; va[4 * i + 2] = x.z; va[4 * i + 3] = x.w;
+        }
+        tmem_st_32x32b_x16(tmem_base + lane_addr + Cfg::kSfaCol0 + 16 * sb, va);
+        uint32_t vb[32];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int g = 0; g < 2; ++g) {
+            const uint4 x = *reinterpret_cast<const uint4*>(sbp + g * GP_SF_TILE + i * 512);
+            vb[8 * i + 4 * g] = x.x; vb[8 * i + 4 * g + 1] = x.y;
+            vb[8 * i + 4 * g + 2] = x.z; vb[8 * i + 4 * g + 3] = x.w;
+          }
+        tmem_st_32x32b_x32(tmem_base + lane_addr + Cfg::kSfbCol0 + 32 * sb, vb);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive_cluster(leader_ready0 + 8 * sb);
+        ++n;
+        if (++stage == S) { stage = 0; phase ^= 1; }
+      }
+    }
   }
 
   // every role of both CTAs is done (remote arrivals delivered, MMAs drained

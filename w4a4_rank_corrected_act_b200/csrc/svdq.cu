@@ -258,8 +258,8 @@ svdq_status gemm_pair_impl(const uint8_t* x_codes, const uint8_t* x_scales, cons
                   static_cast<uint64_t>(r) * 2, rp, 128, lr_swizzle(rp));
     if (s != SVDQ_OK) return s;
   }
-  s = make_tmap(&maps[6], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, N, M, static_cast<uint64_t>(N) * 2, 32, 32,
-                CU_TENSOR_MAP_SWIZZLE_64B);
+  s = make_tmap(&maps[6], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, N, M, static_cast<uint64_t>(N) * 2, 16, 32,
+                CU_TENSOR_MAP_SWIZZLE_32B);
   if (s != SVDQ_OK) return s;
   GemmPairParams p;
   p.bias = w->has_bias ? w->bias : nullptr;
@@ -304,9 +304,9 @@ svdq_status gemm_impl(const uint8_t* x_codes, const uint8_t* x_scales, const uin
   s = make_tmap(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->w_codes, K / 2, N, K / 2, 128, BN,
                 CU_TENSOR_MAP_SWIZZLE_128B);
   if (s != SVDQ_OK) return s;
-  // Y is stored in 32 x 32 pieces through 64-byte-swizzled staging buffers
-  s = make_tmap(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, N, M, static_cast<uint64_t>(N) * 2, 32, 32,
-                CU_TENSOR_MAP_SWIZZLE_64B);
+  // Y is stored in 32-row x 16-column pieces through 32-byte-swizzled staging buffers
+  s = make_tmap(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, N, M, static_cast<uint64_t>(N) * 2, 16, 32,
+                CU_TENSOR_MAP_SWIZZLE_32B);
   if (s != SVDQ_OK) return s;
   if (r > 0) {
     s = make_tmap(&td, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, D, r, M, static_cast<uint64_t>(r) * 2, rp,
