@@ -252,6 +252,24 @@ svdq_status svdq_clear_device_status(void* stream);
  * `stream`; read the result with svdq_get_device_status. */
 svdq_status svdq_selftest_wait_timeout(uint64_t limit_ns, void* stream);
 
+/* Numerics self-test of the activation kernel's quantiser on the current
+ * device (synchronous, default stream).  The kernel takes each element's code
+ * from RN(v / s) computed without a division (one multiply by RN(1/s) and the
+ * FMA quotient correction of Markstein, IBM J. Res. Dev. 34(1), 1990).  This
+ * runs that exact device routine for every E4M3 scale s > 0, both signs, five
+ * binades of v around s and all 2^23 significands of v, plus signed zeros,
+ * subnormal, tiny, huge and tie values for every scale code including s = 0
+ * (whose quotient is defined as a zero with v's sign), and writes
+ * counts[0] = quotients differing from IEEE float32 division where that
+ * quotient is normal or zero, counts[1] = E2M1 codes (sign bit kept)
+ * differing from the format's definition applied to the IEEE quotient, and
+ * counts[2] = quotient differences where the IEEE quotient is subnormal (the
+ * correction step is not exact there, but such quotients lie far below the
+ * first E2M1 threshold 0.25, so their codes are checked by counts[1]).
+ * counts[0] and counts[1] are 0 on a correct build.  `counts` is a host array
+ * of 3.  The paper has no counterpart: this is test support. */
+svdq_status svdq_selftest_quotient(uint64_t* counts);
+
 #ifdef __cplusplus
 }  /* extern "C" */
 #endif

@@ -239,6 +239,34 @@ def test_gemm_parity(M, K, N, r, pair, monkeypatch):
     check_y(to_np_u16(Y), o["Y64"], "gemm")
 
 
+@pytest.mark.parametrize("BN", ["128", "256"])
+def test_gemm_output_16_byte_aligned(BN, monkeypatch):
+    """Y only 16-byte aligned (the interface's minimum): the epilogue's rows go
+    out as two 16-byte stores; rows past M (ragged tail) are never written."""
+    monkeypatch.setenv("SVDQ_GEMM_PAIR", "0")
+    monkeypatch.setenv("SVDQ_GEMM_BN", BN)
+    t = torch()
+    M, K, N, r = 200, 512, 512, 32
+    X, W, B, lam = _inputs(M, K, N, seed=77)
+    lin, exp = _prepare(W, lam, B, r)
+    prep = _oracle_prep_from_export(W, lam, B, exp, r)
+    o = ref.linear_forward(X, prep)
+    codes = dev_u8(o["x_codes"])
+    native = np.zeros(svdq.svdq_act_scales_bytes(M, K), np.uint8)
+    svdq.svdq_scales_to_native(np.ascontiguousarray(o["x_scales"]).ctypes.data, M, K, native.ctypes.data)
+    sc = dev_u8(native)
+    D = dev_u16(o["D"])
+    guard = 0x5A5A
+    buf = t.full((M * N + 64,), guard, dtype=t.int16, device="cuda")
+    Y = buf[8:8 + M * N]                          # 16 bytes past a 256-byte boundary
+    assert Y.data_ptr() % 32 == 16
+    svdq.svdq_gemm(codes.data_ptr(), sc.data_ptr(), D.data_ptr(), M, lin.w, Y.data_ptr(), stream())
+    t.cuda.synchronize()
+    check_y(to_np_u16(Y.view(M, N)), o["Y64"], "gemm, 16-byte aligned Y")
+    rest = to_np_u16(buf)
+    assert np.all(rest[:8] == guard) and np.all(rest[8 + M * N:] == guard)
+
+
 # ---------------------------------------------------------------------------
 # whole layer
 # ---------------------------------------------------------------------------
@@ -313,6 +341,15 @@ def test_empty_and_invalid_calls():
     with pytest.raises(svdq.SvdqError, match="MISALIGNED"):
         svdq.svdq_linear_forward(dev_u16(X).data_ptr() + 2, M, lin.w, Y.data_ptr(), ws.data_ptr(),
                                  lin.workspace_bytes(M), stream())
+
+
+def test_quantiser_quotient_exhaustive():
+    """The activation kernel's division-free quotient equals IEEE division, and
+    its E2M1 codes (sign kept, ties to even) equal the format's definition, for
+    every E4M3 scale and every float32 significand in five binades."""
+    q_bad, c_bad, q_sub = svdq.svdq_selftest_quotient()
+    # subnormal quotients may differ (q_sub), but their codes are checked too
+    assert (q_bad, c_bad) == (0, 0), (q_bad, c_bad, q_sub)
 
 
 def test_device_status_clean():

@@ -63,6 +63,7 @@ SIGNATURES = {
     "svdq_get_device_status": (_I, [_P, ctypes.POINTER(ctypes.c_uint32)]),
     "svdq_clear_device_status": (_I, [_P]),
     "svdq_selftest_wait_timeout": (_I, [ctypes.c_uint64, _P]),
+    "svdq_selftest_quotient": (_I, [ctypes.POINTER(ctypes.c_uint64)]),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -206,6 +207,15 @@ def svdq_clear_device_status(stream: int = 0) -> None:
 
 def svdq_selftest_wait_timeout(limit_ns: int, stream: int = 0) -> None:
     _call("svdq_selftest_wait_timeout", int(limit_ns), stream or None)
+
+
+def svdq_selftest_quotient() -> tuple:
+    """(normal-range quotient mismatches, code mismatches, subnormal-range
+    quotient mismatches) of the activation quantiser's division-free path over
+    its exhaustive sweep; the first two are 0 on a correct build."""
+    out = (ctypes.c_uint64 * 3)()
+    _call("svdq_selftest_quotient", out)
+    return int(out[0]), int(out[1]), int(out[2])
 
 
 # --------------------------------------------------------------------------

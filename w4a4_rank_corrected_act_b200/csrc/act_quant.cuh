@@ -45,7 +45,8 @@ template <int R_PAD>
 struct ActSmem {
   static constexpr uint32_t kRing = ACT_WARPS * ACT_RING * ACT_SUB_BYTES;        // 64 KB
   static constexpr uint32_t kRed = (R_PAD > 0 ? ACT_WARPS * ACT_ROWS * R_PAD * 4 : 0);
-  static constexpr uint32_t kBytes = kRing + kRed + ACT_WARPS * ACT_RING * 8 + 16 + 1024;
+  static constexpr uint32_t kTab = 128 * 8;                                     // E4M3 (s, 1/s)
+  static constexpr uint32_t kBytes = kRing + kRed + kTab + ACT_WARPS * ACT_RING * 8 + 16 + 1024;
 };
 
 // Position (in 32-bit words) of L1 element pair (k, k+1), column j, in the
@@ -67,7 +68,9 @@ __global__ void __launch_bounds__(ACT_THREADS, 2)
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   float* red = reinterpret_cast<float*>(smem + ActSmem<R_PAD>::kRing);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + ActSmem<R_PAD>::kRing + ActSmem<R_PAD>::kRed);
+  float2* tab = reinterpret_cast<float2*>(smem + ActSmem<R_PAD>::kRing + ActSmem<R_PAD>::kRed);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + ActSmem<R_PAD>::kRing + ActSmem<R_PAD>::kRed +
+                                               ActSmem<R_PAD>::kTab);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + ACT_WARPS * ACT_RING);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -88,7 +91,8 @@ __global__ void __launch_bounds__(ACT_THREADS, 2)
     for (int sl = 0; sl < ACT_RING; ++sl) mbar_init(bar(sl), 1);
     fence_mbar_init();
   }
-  __syncthreads();   // barriers and the abort flag are initialised
+  for (int c = threadIdx.x; c < 128; c += ACT_THREADS) tab[c] = e4m3_table_entry(c);
+  __syncthreads();   // barriers, the E4M3 table and the abort flag are initialised
 
   const int my_count = nsub > warp ? (nsub - warp + ACT_WARPS - 1) / ACT_WARPS : 0;
   auto issue = [&](int jj) {
@@ -110,6 +114,14 @@ __global__ void __launch_bounds__(ACT_THREADS, 2)
     for (int i = 0; i < 4; ++i) acc[t][i] = 0.0f;
   const uint32_t half_k = static_cast<uint32_t>(p.K) >> 1;
   const int chunk16 = lane & 7, rsub = lane >> 3;
+  // 1/lambda of this lane's 8 columns, one sub-tile ahead
+  float4 ni0 = make_float4(0.f, 0.f, 0.f, 0.f), ni1 = ni0;
+  auto load_inv = [&](int j) {
+    const float* src = p.inv_lambda + (warp + ACT_WARPS * j) * ACT_SUB + 8 * chunk16;
+    ni0 = __ldg(reinterpret_cast<const float4*>(src));
+    ni1 = __ldg(reinterpret_cast<const float4*>(src + 4));
+  };
+  if (my_count > 0) load_inv(0);
   int jj = 0;
   for (; jj < my_count; ++jj) {
     const int slot = jj % ACT_RING;
@@ -125,9 +137,10 @@ __global__ void __launch_bounds__(ACT_THREADS, 2)
           if (t < nt_count)
             bfr[ks][t] = __ldg(f + ((static_cast<size_t>(col0 / 16 + ks) * nt_count + t) * 32 + lane));
     }
-    const float4 i0 = __ldg(reinterpret_cast<const float4*>(p.inv_lambda + col0 + 8 * chunk16));
-    const float4 i1 = __ldg(reinterpret_cast<const float4*>(p.inv_lambda + col0 + 8 * chunk16 + 4));
-    const float inv[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
+    // -1/lambda: the quantiser takes -Xhat (see nvfp4_quant_half_block_x2)
+    const uint64_t ninv2[4] = {f32x2_pack(-ni0.x, -ni0.y), f32x2_pack(-ni0.z, -ni0.w),
+                               f32x2_pack(-ni1.x, -ni1.y), f32x2_pack(-ni1.z, -ni1.w)};
+    if (jj + 1 < my_count) load_inv(jj + 1);
     if (!mbar_wait(bar(slot), (jj / ACT_RING) & 1, abort_flag, KID_ACT, 1)) break;
     uint8_t* tile = smem + (ring - smem_u32(smem)) + slot * ACT_SUB_BYTES;
 
@@ -138,14 +151,15 @@ __global__ void __launch_bounds__(ACT_THREADS, 2)
       const uint32_t off = swz(row * 128 + chunk16 * 16, 3);
       const uint4 raw = *reinterpret_cast<const uint4*>(tile + off);
       const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
-      float xh[8];
+      // -Xhat = f32(x * (-1/lambda)) (exactly the negated product), element 2u
+      // in the low half of pair u
+      uint64_t nxh[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        xh[2 * u] = __fmul_rn(bf16_bits_to_f32(w4[u] & 0xFFFFu), inv[2 * u]);
-        xh[2 * u + 1] = __fmul_rn(bf16_bits_to_f32(w4[u] >> 16), inv[2 * u + 1]);
-      }
+      for (int u = 0; u < 4; ++u)
+        nxh[u] = f32x2_mul(f32x2_pack(__uint_as_float(w4[u] << 16), __uint_as_float(w4[u] & 0xFFFF0000u)),
+                           ninv2[u]);
       uint32_t sc;
-      const uint32_t codes = nvfp4_quant_half_block(xh, sc);
+      const uint32_t codes = nvfp4_quant_half_block_x2(nxh, tab, sc);
       if (grow < p.M)
         *reinterpret_cast<uint32_t*>(p.x_codes + static_cast<size_t>(grow) * half_k +
                                      (col0 >> 1) + 4 * chunk16) = codes;
@@ -157,12 +171,16 @@ __global__ void __launch_bounds__(ACT_THREADS, 2)
         *reinterpret_cast<uint32_t*>(p.x_scales + sf_offset(grow, col0 >> 4, p.K)) =
             sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
       if (R_PAD > 0) {
-        uint4 o;
-        o.x = pack_bf16x2(xh[0], xh[1]);
-        o.y = pack_bf16x2(xh[2], xh[3]);
-        o.z = pack_bf16x2(xh[4], xh[5]);
-        o.w = pack_bf16x2(xh[6], xh[7]);
-        *reinterpret_cast<uint4*>(tile + off) = o;
+        // bf16(-Xhat) = -bf16(Xhat): the tile holds the negated operand, and the
+        // product with L1 is negated back when D is written
+        uint32_t o[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          float lo, hi;
+          f32x2_unpack(nxh[u], lo, hi);
+          o[u] = pack_bf16x2(lo, hi);
+        }
+        *reinterpret_cast<uint4*>(tile + off) = make_uint4(o[0], o[1], o[2], o[3]);
       }
     }
 
@@ -209,7 +227,7 @@ __global__ void __launch_bounds__(ACT_THREADS, 2)
         float v = 0.0f;
 #pragma unroll
         for (int w = 0; w < ACT_WARPS; ++w) v += red[(w * ACT_ROWS + row) * R_PAD + col];
-        p.D[static_cast<size_t>(grow) * p.r + col] = static_cast<uint16_t>(pack_bf16x2(v, 0.0f) & 0xFFFFu);
+        p.D[static_cast<size_t>(grow) * p.r + col] = static_cast<uint16_t>(pack_bf16x2(-v, 0.0f) & 0xFFFFu);
       }
     }
   }

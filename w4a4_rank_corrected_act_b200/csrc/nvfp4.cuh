@@ -101,6 +101,85 @@ __device__ __forceinline__ uint32_t nvfp4_quant_half_block(const float (&v)[8],
   return e2m1x8_magnitudes(mag) | signs;
 }
 
+// Packed float32 pairs (Blackwell f32x2 arithmetic, each half an ordinary
+// IEEE round-to-nearest-even operation).
+__device__ __forceinline__ uint64_t f32x2_pack(float lo, float hi) {
+  uint64_t d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+  return d;
+}
+__device__ __forceinline__ void f32x2_unpack(uint64_t d, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(d));
+}
+__device__ __forceinline__ uint64_t f32x2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f32x2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+// Entry c of the E4M3 table: (s, RN(1/s)) for s = E4M3 value of code c, and
+// (0, 0) for c == 0.
+__device__ __forceinline__ float2 e4m3_table_entry(uint32_t c) {
+  const float s = e4m3_to_f32(c);
+  return make_float2(s, s == 0.0f ? 0.0f : __frcp_rn(s));
+}
+
+// Correctly rounded quotients v / s of a pair, without a division, by the
+// quotient-correction step of Markstein (IBM J. Res. Dev. 34(1), 1990, "Computation
+// of elementary functions on the IBM RISC System/6000 processor"): with
+// y = RN(1/s) and q0 = RN(v y) (faithful), the remainder v - s q0 is exact in
+// one FMA and RN(q0 + (v - s q0) y) = RN(v / s).
+// The input is u = -v (the pair negated) and the constants are s2 = (s, s) and
+// neg_y2 = (-y, -y): then q0 = u (-y), rn = s q0 + u = -(v - s q0) and the
+// result is q0 + rn (-y).  Every step is the textbook one up to exact
+// negations, and a zero v gives a zero quotient with v's sign (-0 / s = -0):
+// the plain ordering would return +0 for v = -0, since the exact remainder
+// +0 + (-0) rounds to +0.  With s = y = 0 the result is a zero with v's sign.
+__device__ __forceinline__ uint64_t quotient_f32x2(uint64_t u, uint64_t s2, uint64_t neg_y2) {
+  const uint64_t q0 = f32x2_mul(u, neg_y2);
+  const uint64_t rn = f32x2_fma(s2, q0, u);
+  return f32x2_fma(rn, neg_y2, q0);
+}
+
+// E2M1 codes (RNE, satfinite, sign kept) of the 8 signed floats q0..q7, q0 in
+// the lowest nibble.
+__device__ __forceinline__ uint32_t e2m1x8_signed(const uint64_t (&q)[4]) {
+  float a[8];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) f32x2_unpack(q[u], a[2 * u], a[2 * u + 1]);
+  return e2m1x8_magnitudes(a);
+}
+
+// Same result as nvfp4_quant_half_block for the 8 values v, given NEGATED and
+// packed in pairs (nv[u] = (-v[2u], -v[2u+1])), taking s and RN(1/s) from
+// `tab` (128 entries of e4m3_table_entry, in shared memory) and the codes from
+// the correctly rounded quotients of quotient_f32x2.  Called by all 32 lanes;
+// the other half of the block lives on lane (laneid ^ 1).
+__device__ __forceinline__ uint32_t nvfp4_quant_half_block_x2(const uint64_t (&nv)[4], const float2* tab,
+                                                             uint32_t& scale_code) {
+  float am = 0.0f;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    float lo, hi;
+    f32x2_unpack(nv[u], lo, hi);
+    am = fmaxf(am, fmaxf(fabsf(lo), fabsf(hi)));
+  }
+  am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+  const uint32_t sc = e4m3_rn_satfinite(__fdiv_rn(am, 6.0f));
+  scale_code = sc;
+  const float2 sy = tab[sc];
+  const uint64_t s2 = f32x2_pack(sy.x, sy.x), neg_y2 = f32x2_pack(-sy.y, -sy.y);
+  uint64_t q[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) q[u] = quotient_f32x2(nv[u], s2, neg_y2);
+  return e2m1x8_signed(q);
+}
+
 // Byte offset of scale (row, kb16) in the scale-factor tile layout:
 // 512-byte tiles of 128 rows x 4 scales, tile (row/128, kb16/4) at
 // ((row/128) * (K/64) + kb16/4) * 512, inside it (row%32)*16 + ((row/32)%4)*4 + kb16%4.

@@ -304,7 +304,6 @@ svdq_status gemm_impl(const uint8_t* x_codes, const uint8_t* x_scales, const uin
   s = make_tmap(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->w_codes, K / 2, N, K / 2, 128, BN,
                 CU_TENSOR_MAP_SWIZZLE_128B);
   if (s != SVDQ_OK) return s;
-  // Y is stored in 32-row x 16-column pieces through 32-byte-swizzled staging buffers
   s = make_tmap(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, N, M, static_cast<uint64_t>(N) * 2, 16, 32,
                 CU_TENSOR_MAP_SWIZZLE_32B);
   if (s != SVDQ_OK) return s;
@@ -316,7 +315,7 @@ svdq_status gemm_impl(const uint8_t* x_codes, const uint8_t* x_scales, const uin
                   static_cast<uint64_t>(r) * 2, rp, BN, lr_swizzle(rp));
     if (s != SVDQ_OK) return s;
   }
-  GemmParams p;
+  GemmParams p{};
   p.x_scales = x_scales;
   p.w_scales = w->w_scales;
   p.bias = w->has_bias ? w->bias : nullptr;
@@ -451,6 +450,65 @@ __global__ void selftest_wait_kernel(unsigned long long limit_ns) {
     mbar_wait(smem_u32(&bar), 0, reinterpret_cast<volatile int*>(&abort_flag), KID_SELFTEST, 1,
               limit_ns);
   __syncthreads();
+}
+
+// Exhaustive check of the activation kernel's division-free quotient
+// (quotient_f32x2) and of the E2M1 conversion of its signed result.  For every
+// positive E4M3 scale s (codes 1..126), both signs, five binades of v around s
+// (v / s in [1/8, 8)) and all 2^23 significands of v -- plus zeros, subnormal,
+// tiny and huge v for every code including s = 0 -- count quotients that
+// differ from IEEE division (counts[0] where the IEEE quotient is a normal
+// number or zero, counts[2] where it is subnormal, a range in which the
+// correction step is not exact; for s = 0 the defined quotient is a zero with
+// v's sign) and codes that differ from E2M1 of the IEEE quotient by the
+// format's definition (counts[1]): magnitude thresholds 0.25, 0.75, 1.25,
+// 1.75, 2.5, 3.5, 5 with ties to the even code, sign kept.
+__device__ unsigned long long g_quotient_mismatch[3];
+
+__device__ void check_quotient(uint32_t c, float v) {
+  const float thr[7] = {0.25f, 0.75f, 1.25f, 1.75f, 2.5f, 3.5f, 5.0f};
+  const float2 sy = e4m3_table_entry(c);
+  const float qr = c == 0 ? __uint_as_float(__float_as_uint(v) & 0x80000000u) : __fdiv_rn(v, sy.x);
+  float qt, qt2;
+  f32x2_unpack(quotient_f32x2(f32x2_pack(-v, -v), f32x2_pack(sy.x, sy.x), f32x2_pack(-sy.y, -sy.y)), qt,
+               qt2);
+  if (__float_as_uint(qt) != __float_as_uint(qr) || __float_as_uint(qt2) != __float_as_uint(qr)) {
+    const bool subnormal = qr != 0.0f && fabsf(qr) < 0x1p-126f;
+    atomicAdd(&g_quotient_mismatch[subnormal ? 2 : 0], 1ull);
+  }
+  const float a[8] = {qt, qt, qt, qt, qt, qt, qt, qt};
+  const uint32_t got = e2m1x8_magnitudes(a) & 15u;
+  const float mag = fabsf(qr);
+  uint32_t want = 0;
+#pragma unroll
+  for (int k = 0; k < 7; ++k)
+    if (mag > thr[k] || (mag == thr[k] && (k & 1))) want = static_cast<uint32_t>(k + 1);
+  want |= (__float_as_uint(qr) >> 31) << 3;
+  if (got != want) atomicAdd(&g_quotient_mismatch[1], 1ull);
+}
+
+__global__ void selftest_quotient_kernel() {
+  const unsigned long long total = 126ull * 5ull * 2ull << 23;
+  for (unsigned long long idx = static_cast<unsigned long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+       idx < total; idx += static_cast<unsigned long long>(gridDim.x) * blockDim.x) {
+    const uint32_t m = static_cast<uint32_t>(idx) & ((1u << 23) - 1u);
+    unsigned long long rest = idx >> 23;
+    const uint32_t neg = static_cast<uint32_t>(rest & 1ull);
+    rest >>= 1;
+    const int d = static_cast<int>(rest % 5ull) - 2;
+    const uint32_t c = 1u + static_cast<uint32_t>(rest / 5ull);
+    const int es = static_cast<int>((__float_as_uint(e4m3_to_f32(c)) >> 23) & 255u);
+    check_quotient(c, __uint_as_float((neg << 31) | (static_cast<uint32_t>(es + d) << 23) | m));
+  }
+  if (blockIdx.x == 0) {
+    // zeros, smallest subnormal, smallest normal, tiny, huge, exact ties
+    const uint32_t special[10] = {0x00000000u, 0x00000001u, 0x00800000u, 0x0DA24260u, 0x45BB8000u,
+                                  0x3E99999Au, 0x40200000u, 0x33D6BF95u, 0x3E800000u, 0x40A00000u};
+    for (int t = threadIdx.x; t < 127 * 20; t += blockDim.x) {
+      const uint32_t c = static_cast<uint32_t>(t / 20), j = static_cast<uint32_t>(t % 20);
+      check_quotient(c, __uint_as_float(special[j >> 1] | ((j & 1u) << 31)));
+    }
+  }
 }
 
 // --------------------------------------------------------------------------
@@ -772,6 +830,19 @@ svdq_status svdq_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
       std::min<unsigned long long>(std::max<unsigned long long>(limit_ns, 1000ull), 1000000000ull);
   selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(lim);
   SVDQ_CHECK_LAUNCH("selftest_wait_kernel");
+  return SVDQ_OK;
+}
+
+svdq_status svdq_selftest_quotient(uint64_t* counts) {
+  if (counts == nullptr) return SVDQ_ERR_INVALID_ARG;
+  const unsigned long long z[3] = {0ull, 0ull, 0ull};
+  SVDQ_CUDA(cudaMemcpyToSymbol(g_quotient_mismatch, z, sizeof(z)));
+  selftest_quotient_kernel<<<num_sms() * 8, 256>>>();
+  SVDQ_CHECK_LAUNCH("selftest_quotient_kernel");
+  SVDQ_CUDA(cudaDeviceSynchronize());
+  unsigned long long out[3];
+  SVDQ_CUDA(cudaMemcpyFromSymbol(out, g_quotient_mismatch, sizeof(out)));
+  for (int i = 0; i < 3; ++i) counts[i] = out[i];
   return SVDQ_OK;
 }
 
