@@ -122,6 +122,22 @@ __global__ void __launch_bounds__(ACT_THREADS, 2)
     ni1 = __ldg(reinterpret_cast<const float4*>(src + 4));
   };
   if (my_count > 0) load_inv(0);
+  const float y6 = tab[0x4C].y;   // E4M3 code 0x4C is 6.0: RN(1/6)
+  const uint64_t six = f32x2_pack(6.0f, 6.0f), neg_y6 = f32x2_pack(-y6, -y6);
+  // row-dependent addresses, fixed for the whole K range: the 16 bytes of
+  // row 4 i + l / 8 in a (swizzled) sub-tile, its codes (null past M) and its
+  // scale bytes of column group 0 (one byte per 16-element block, written by
+  // the lower lane of each pair)
+  uint32_t toff[ACT_ROWS / 4];
+  uint8_t* cptr[ACT_ROWS / 4];
+  uint8_t* sptr[ACT_ROWS / 4];
+#pragma unroll
+  for (int i = 0; i < ACT_ROWS / 4; ++i) {
+    const int row = i * 4 + rsub, grow = row0 + row;
+    toff[i] = swz(static_cast<uint32_t>(row * 128 + chunk16 * 16), 3);
+    cptr[i] = grow < p.M ? p.x_codes + static_cast<size_t>(grow) * half_k + 4 * chunk16 : nullptr;
+    sptr[i] = p.x_scales + sf_offset(static_cast<uint32_t>(grow), 0, static_cast<uint32_t>(p.K)) + chunk16 / 2;
+  }
   int jj = 0;
   for (; jj < my_count; ++jj) {
     const int slot = jj % ACT_RING;
@@ -146,9 +162,7 @@ __global__ void __launch_bounds__(ACT_THREADS, 2)
 
 #pragma unroll
     for (int i = 0; i < ACT_ROWS / 4; ++i) {
-      const int row = i * 4 + rsub;
-      const int grow = row0 + row;
-      const uint32_t off = swz(row * 128 + chunk16 * 16, 3);
+      const uint32_t off = toff[i];
       const uint4 raw = *reinterpret_cast<const uint4*>(tile + off);
       const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
       // -Xhat = f32(x * (-1/lambda)) (exactly the negated product), element 2u
@@ -159,17 +173,9 @@ __global__ void __launch_bounds__(ACT_THREADS, 2)
         nxh[u] = f32x2_mul(f32x2_pack(__uint_as_float(w4[u] << 16), __uint_as_float(w4[u] & 0xFFFF0000u)),
                            ninv2[u]);
       uint32_t sc;
-      const uint32_t codes = nvfp4_quant_half_block_x2(nxh, tab, sc);
-      if (grow < p.M)
-        *reinterpret_cast<uint32_t*>(p.x_codes + static_cast<size_t>(grow) * half_k +
-                                     (col0 >> 1) + 4 * chunk16) = codes;
-      // the 4 scales of this row's 64 columns sit on lanes 8a, 8a+2, 8a+4, 8a+6
-      const uint32_t s1 = __shfl_down_sync(0xffffffffu, sc, 2);
-      const uint32_t s2 = __shfl_down_sync(0xffffffffu, sc, 4);
-      const uint32_t s3 = __shfl_down_sync(0xffffffffu, sc, 6);
-      if (chunk16 == 0)
-        *reinterpret_cast<uint32_t*>(p.x_scales + sf_offset(grow, col0 >> 4, p.K)) =
-            sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
+      const uint32_t codes = nvfp4_quant_half_block_x2(nxh, tab, six, neg_y6, sc);
+      if (cptr[i] != nullptr) *reinterpret_cast<uint32_t*>(cptr[i] + (col0 >> 1)) = codes;
+      if ((chunk16 & 1) == 0) sptr[i][static_cast<size_t>(col0 >> 6) * 512] = static_cast<uint8_t>(sc);
       if (R_PAD > 0) {
         // bf16(-Xhat) = -bf16(Xhat): the tile holds the negated operand, and the
         // product with L1 is negated back when D is written

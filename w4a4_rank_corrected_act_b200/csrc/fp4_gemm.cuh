@@ -228,10 +228,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
     mbar_init(tmem_full(0), 1);
     mbar_init(tmem_full(1), 1);
-    mbar_init(tmem_free, 128);
+    mbar_init(tmem_free, 4);          // one arrive per epilogue warp
     mbar_init(drain_bar, 1);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(sf_ready(b), 128);
+      mbar_init(sf_ready(b), 4);      // one arrive per scale warp
       mbar_init(sf_free(b), 1);
     }
     *abort_flag = 0;
@@ -387,7 +387,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       epilogue_tile<BN, kOv>(
           acc, lane_addr, lane, p.bias != nullptr, tile_bias, n0, m0 + q * 32, &tm_y, stg, stg_u,
           [&](int i) { return buf ? i : (i + kPieces - kOv) % kPieces; },
-          [&]() { mbar_arrive(tmem_free); });
+          [&]() {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tmem_free);
+          });
     }
     if (lane == 0) bulk_wait_group_all();
     __syncwarp();
@@ -408,12 +411,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       }
       for (int kb = 0; kb < kb_per_tile; ++kb) {
         if (!mbar_wait(full_bar(stage), phase, abort_flag, KID_GEMM, 20)) { ok = false; break; }
-        const uint32_t sb = n & 1u;
-        if (n >= 2 && !mbar_wait(sf_free(sb), ((n >> 1) - 1) & 1u, abort_flag, KID_GEMM, 21)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
         const uint8_t* sa = smem + (stage_sfa(stage) - smem_base) + lane * 16;
         const uint8_t* sbp = smem + (stage_sfb(stage) - smem_base) + lane * 16;
         uint32_t va[16];
@@ -422,30 +419,29 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           const uint4 x = *reinterpret_cast<const uint4*>(sa + i * 512);
           va[4 * i] = x.x; va[4 * i + 1] = x.y; va[4 * i + 2] = x.z; va[4 * i + 3] = x.w;
         }
-        tmem_st_32x32b_x16(tmem_base + lane_addr + Cfg::kSfaCol0 + 16 * sb, va);
-        if (BN == 256) {
-          uint32_t vb[32];
+        constexpr int kG = BN / 128;
+        uint32_t vb[16 * kG];
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
+        for (int i = 0; i < 4; ++i)
 #pragma unroll
-            for (int g = 0; g < 2; ++g) {
-              const uint4 x = *reinterpret_cast<const uint4*>(sbp + (g * 4 + i) * 512);
-              vb[8 * i + 4 * g] = x.x; vb[8 * i + 4 * g + 1] = x.y;
-              vb[8 * i + 4 * g + 2] = x.z; vb[8 * i + 4 * g + 3] = x.w;
-            }
-          tmem_st_32x32b_x32(tmem_base + lane_addr + Cfg::kSfbCol0 + 32 * sb, vb);
-        } else {
-          uint32_t vb[16];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint4 x = *reinterpret_cast<const uint4*>(sbp + i * 512);
-            vb[4 * i] = x.x; vb[4 * i + 1] = x.y; vb[4 * i + 2] = x.z; vb[4 * i + 3] = x.w;
+          for (int g = 0; g < kG; ++g) {
+            const uint4 x = *reinterpret_cast<const uint4*>(sbp + (g * 4 + i) * 512);
+            vb[4 * kG * i + 4 * g] = x.x; vb[4 * kG * i + 4 * g + 1] = x.y;
+            vb[4 * kG * i + 4 * g + 2] = x.z; vb[4 * kG * i + 4 * g + 3] = x.w;
           }
-          tmem_st_32x32b_x16(tmem_base + lane_addr + Cfg::kSfbCol0 + 32 * sb, vb);
+        const uint32_t sb = n & 1u;
+        if (n >= 2 && !mbar_wait(sf_free(sb), ((n >> 1) - 1) & 1u, abort_flag, KID_GEMM, 21)) {
+          ok = false;
+          break;
         }
+        tc_fence_after();
+        tmem_st_32x32b_x16(tmem_base + lane_addr + Cfg::kSfaCol0 + 16 * sb, va);
+        if constexpr (kG == 2) tmem_st_32x32b_x32(tmem_base + lane_addr + Cfg::kSfbCol0 + 32 * sb, vb);
+        else tmem_st_32x32b_x16(tmem_base + lane_addr + Cfg::kSfbCol0 + 32 * sb, vb);
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(sf_ready(sb));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sf_ready(sb));
         ++n;
         if (++stage == S) { stage = 0; phase ^= 1; }
       }

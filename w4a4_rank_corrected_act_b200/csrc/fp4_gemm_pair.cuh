@@ -109,10 +109,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GP_THREADS, 1)
     }
     mbar_init(tmem_full(0), 1);
     mbar_init(tmem_full(1), 1);
-    mbar_init(tmem_free, 2 * 128);    // both CTAs' epilogue threads
+    mbar_init(tmem_free, 2 * 4);      // both CTAs' epilogue warps
     mbar_init(drain_bar, 1);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(sf_ready(b), 2 * 128);  // both CTAs' scale warps
+      mbar_init(sf_ready(b), 2 * 4);  // both CTAs' scale warps
       mbar_init(sf_free(b), 1);         // one multicast MMA commit
     }
     for (int st = 0; st < S; ++st) mbar_init(sf_full(st), 1);
@@ -275,7 +275,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GP_THREADS, 1)
       epilogue_tile<GP_BN, kOv>(
           acc, lane_addr, lane, p.bias != nullptr, tile_bias, n0, m0 + q * 32, &tm_y, stg, stg_u,
           [&](int i) { return buf ? i : (i + kPieces - kOv) % kPieces; },
-          [&]() { mbar_arrive_cluster(leader_free); });
+          [&]() {
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(leader_free);
+          });
     }
     if (lane == 0) bulk_wait_group_all();
     __syncwarp();
@@ -321,7 +324,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GP_THREADS, 1)
         tmem_st_32x32b_x32(tmem_base + lane_addr + Cfg::kSfbCol0 + 32 * sb, vb);
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive_cluster(leader_ready0 + 8 * sb);
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(leader_ready0 + 8 * sb);
         ++n;
         if (++stage == S) { stage = 0; phase ^= 1; }
       }

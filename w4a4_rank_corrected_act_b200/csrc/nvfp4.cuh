@@ -157,10 +157,12 @@ __device__ __forceinline__ uint32_t e2m1x8_signed(const uint64_t (&q)[4]) {
 
 // Same result as nvfp4_quant_half_block for the 8 values v, given NEGATED and
 // packed in pairs (nv[u] = (-v[2u], -v[2u+1])), taking s and RN(1/s) from
-// `tab` (128 entries of e4m3_table_entry, in shared memory) and the codes from
-// the correctly rounded quotients of quotient_f32x2.  Called by all 32 lanes;
-// the other half of the block lives on lane (laneid ^ 1).
+// `tab` (128 entries of e4m3_table_entry, in shared memory) and every
+// quotient -- amax / 6 as well as the element quotients -- from
+// quotient_f32x2 (six = (6, 6), neg_y6 = (-RN(1/6), -RN(1/6))).  Called by
+// all 32 lanes; the other half of the block lives on lane (laneid ^ 1).
 __device__ __forceinline__ uint32_t nvfp4_quant_half_block_x2(const uint64_t (&nv)[4], const float2* tab,
+                                                             uint64_t six, uint64_t neg_y6,
                                                              uint32_t& scale_code) {
   float am = 0.0f;
 #pragma unroll
@@ -170,7 +172,9 @@ __device__ __forceinline__ uint32_t nvfp4_quant_half_block_x2(const uint64_t (&n
     am = fmaxf(am, fmaxf(fabsf(lo), fabsf(hi)));
   }
   am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
-  const uint32_t sc = e4m3_rn_satfinite(__fdiv_rn(am, 6.0f));
+  float a6, a6b;
+  f32x2_unpack(quotient_f32x2(f32x2_pack(-am, -am), six, neg_y6), a6, a6b);   // RN(amax / 6)
+  const uint32_t sc = e4m3_rn_satfinite(a6);
   scale_code = sc;
   const float2 sy = tab[sc];
   const uint64_t s2 = f32x2_pack(sy.x, sy.x), neg_y2 = f32x2_pack(-sy.y, -sy.y);
