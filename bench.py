@@ -41,8 +41,10 @@ UNIT = "TFLOP/s"
 FP4_SPEC_TFLOPS = 9000.0          # dense NVFP4, NVIDIA B200 datasheet
 FP4_OVER_BF16 = 4.0               # nominal dense ratio fp4 : bf16 (9 / 2.25 PFLOP/s)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-GEMM_SRC = os.path.join(ROOT, "w4a4_rank_corrected_act_b200", "csrc", "fp4_gemm.cuh")
-ACT_SRC = os.path.join(ROOT, "w4a4_rank_corrected_act_b200", "csrc", "act_quant.cuh")
+_CSRC = os.path.join(ROOT, "w4a4_rank_corrected_act_b200", "csrc")
+# the sources each kernel is compiled from (a profile is stale once any changed)
+GEMM_SRC = [os.path.join(_CSRC, f) for f in ("fp4_gemm.cuh", "ptx.cuh", "nvfp4.cuh")]
+ACT_SRC = [os.path.join(_CSRC, f) for f in ("act_quant.cuh", "ptx.cuh", "nvfp4.cuh")]
 
 
 def _peaks():
@@ -55,9 +57,12 @@ def _peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def _src_sha(path: str) -> str:
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+def _src_sha(paths) -> str:
+    h = hashlib.sha256()
+    for path in paths:
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def _profile_traffic(kernel_src: str, name: str):
