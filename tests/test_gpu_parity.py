@@ -128,6 +128,19 @@ def _oracle_prep_from_export(W, lam, bias, exp, r):
 @pytest.mark.parametrize("M,K,r", [(256, 512, 32), (1, 256, 16), (17, 768, 32), (129, 512, 64),
                                    (300, 1024, 8), (64, 256, 0), (200, 512, 48)])
 def test_act_quant_parity(M, K, r):
+    _act_parity_case(M, K, r)
+
+
+@pytest.mark.parametrize("ks", [1, 2, 3, 4, 6, 8])
+@pytest.mark.parametrize("r", [32, 64, 0])
+def test_act_quant_parity_k_split(ks, r, monkeypatch):
+    """Clusters of ks CTAs sharing each 16-row block (the small-M path), each
+    CTA one of ks equal K ranges, partial D summed in the first CTA."""
+    monkeypatch.setenv("SVDQ_ACT_KS", str(ks))
+    _act_parity_case(40, 3072, r)
+
+
+def _act_parity_case(M, K, r):
     X, W, _, lam = _inputs(M, K, max(128, r), seed=M * 7 + K + r)
     inv = ref.inv_lambda_of(lam)
     rng = np.random.default_rng(5)

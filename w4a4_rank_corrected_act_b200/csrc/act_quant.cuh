@@ -11,7 +11,10 @@
 //     section "Under the Hood": the low-rank correction runs in higher precision).
 //
 // Design (B200): a CTA owns 16 token rows (one m16 tile); its 8 warps split K
-// into 64-column sub-tiles (warp w takes sub-tiles w, w+8, ...).  Each warp
+// into 64-column sub-tiles (warp w takes sub-tiles w, w+8, ...).  When there
+// are too few rows to fill the GPU, a cluster of ks CTAs shares a row block,
+// CTA c taking the c-th of ks equal K ranges; their partial D meet in the
+// first CTA's shared memory.  Each warp
 // streams its sub-tiles through a private 4-slot TMA ring (16 x 64 bf16 boxes,
 // 128-byte swizzle), so no block-wide synchronisation happens until the final
 // reduction of D.  In a slot, lane pairs quantise 16-element blocks in
@@ -31,6 +34,7 @@ constexpr int ACT_THREADS = ACT_WARPS * 32;
 constexpr int ACT_SUB = 64;           // columns per sub-tile
 constexpr int ACT_RING = 4;           // slots per warp
 constexpr uint32_t ACT_SUB_BYTES = ACT_ROWS * ACT_SUB * 2;   // 2 KB
+constexpr int ACT_MAX_KS = 8;         // CTAs per cluster (K split), portable limit
 
 struct ActParams {
   const float* inv_lambda;
@@ -39,6 +43,7 @@ struct ActParams {
   uint8_t* x_scales;
   uint16_t* D;
   int M, K, r, M_pad;
+  int ks;                  // CTAs per cluster sharing a row block (K split); K % (64 ks) == 0
 };
 
 template <int R_PAD>
@@ -47,6 +52,9 @@ struct ActSmem {
   static constexpr uint32_t kRed = (R_PAD > 0 ? ACT_WARPS * ACT_ROWS * R_PAD * 4 : 0);
   static constexpr uint32_t kTab = 128 * 8;                                     // E4M3 (s, 1/s)
   static constexpr uint32_t kBytes = kRing + kRed + kTab + ACT_WARPS * ACT_RING * 8 + 16 + 1024;
+  // with a K split, the partial D of each CTA of a cluster is gathered in the
+  // first CTA's ring, [rank][row][col], once every CTA is done with its ring
+  static_assert(ACT_MAX_KS * ACT_ROWS * R_PAD * 4 <= kRing, "partial-D gather area");
 };
 
 // Position (in 32-bit words) of L1 element pair (k, k+1), column j, in the
@@ -69,17 +77,21 @@ __global__ void __launch_bounds__(ACT_THREADS, 2)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   float* red = reinterpret_cast<float*>(smem + ActSmem<R_PAD>::kRing);
   float2* tab = reinterpret_cast<float2*>(smem + ActSmem<R_PAD>::kRing + ActSmem<R_PAD>::kRed);
+  float* recv = reinterpret_cast<float*>(smem);   // aliases the ring (see ActSmem)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + ActSmem<R_PAD>::kRing + ActSmem<R_PAD>::kRed +
                                                ActSmem<R_PAD>::kTab);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + ACT_WARPS * ACT_RING);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row0 = blockIdx.x * ACT_ROWS;
-  const int nsub = p.K / ACT_SUB;
+  const uint32_t kpart = p.ks > 1 ? cluster_ctarank() : 0u;
+  const int row0 = (blockIdx.x / p.ks) * ACT_ROWS;
+  const int nsub = p.K / ACT_SUB / p.ks;             // sub-tiles of this CTA's K range
+  const int sub0 = static_cast<int>(kpart) * nsub;   // its first sub-tile
   if (row0 >= p.M) {
     // rows entirely in [M, M_pad): their scale entries are written as zero
+    // (the whole cluster shares the row block, so every CTA of it leaves here)
     for (int idx = threadIdx.x; idx < nsub * ACT_ROWS; idx += ACT_THREADS) {
-      const int g = idx / ACT_ROWS, i = idx % ACT_ROWS;
+      const int g = sub0 + idx / ACT_ROWS, i = idx % ACT_ROWS;
       *reinterpret_cast<uint32_t*>(p.x_scales + sf_offset(row0 + i, g * 4, p.K)) = 0u;
     }
     return;
@@ -98,7 +110,7 @@ __global__ void __launch_bounds__(ACT_THREADS, 2)
   auto issue = [&](int jj) {
     const int slot = jj % ACT_RING;
     mbar_arrive_expect_tx(bar(slot), ACT_SUB_BYTES);
-    tma_load_2d(ring + slot * ACT_SUB_BYTES, &tm_x, bar(slot), (warp + ACT_WARPS * jj) * ACT_SUB,
+    tma_load_2d(ring + slot * ACT_SUB_BYTES, &tm_x, bar(slot), (sub0 + warp + ACT_WARPS * jj) * ACT_SUB,
                 row0);
   };
   if (lane == 0) {
@@ -117,7 +129,7 @@ __global__ void __launch_bounds__(ACT_THREADS, 2)
   // 1/lambda of this lane's 8 columns, one sub-tile ahead
   float4 ni0 = make_float4(0.f, 0.f, 0.f, 0.f), ni1 = ni0;
   auto load_inv = [&](int j) {
-    const float* src = p.inv_lambda + (warp + ACT_WARPS * j) * ACT_SUB + 8 * chunk16;
+    const float* src = p.inv_lambda + (sub0 + warp + ACT_WARPS * j) * ACT_SUB + 8 * chunk16;
     ni0 = __ldg(reinterpret_cast<const float4*>(src));
     ni1 = __ldg(reinterpret_cast<const float4*>(src + 4));
   };
@@ -141,7 +153,7 @@ __global__ void __launch_bounds__(ACT_THREADS, 2)
   int jj = 0;
   for (; jj < my_count; ++jj) {
     const int slot = jj % ACT_RING;
-    const int col0 = (warp + ACT_WARPS * jj) * ACT_SUB;
+    const int col0 = (sub0 + warp + ACT_WARPS * jj) * ACT_SUB;
     // B fragments of this sub-tile's 4 k-steps (L2-resident), issued early
     uint2 bfr[4][kNT > 0 ? kNT : 1];
     if (R_PAD > 0) {
@@ -225,15 +237,43 @@ __global__ void __launch_bounds__(ACT_THREADS, 2)
       mine[(rlo + 8) * R_PAD + col + 1] = acc[t][3];
     }
     __syncthreads();
-    if (!*abort_flag) {
+    if (p.ks == 1) {
+      if (!*abort_flag) {
+        for (int idx = threadIdx.x; idx < ACT_ROWS * p.r; idx += ACT_THREADS) {
+          const int row = idx / p.r, col = idx % p.r;
+          const int grow = row0 + row;
+          if (grow >= p.M) continue;
+          float v = 0.0f;
+#pragma unroll
+          for (int w = 0; w < ACT_WARPS; ++w) v += red[(w * ACT_ROWS + row) * R_PAD + col];
+          p.D[static_cast<size_t>(grow) * p.r + col] = static_cast<uint16_t>(pack_bf16x2(-v, 0.0f) & 0xFFFFu);
+        }
+      }
+    } else {
+      // this CTA's partial (summed over its warps) goes to the first CTA of the
+      // cluster, which adds the ks partials in rank order and writes D; the
+      // first barrier makes sure that CTA no longer uses its ring
+      __syncwarp();
+      cluster_sync_all();
+      const uint32_t dst0 = mapa_shared(smem_u32(recv), 0) + kpart * (ACT_ROWS * R_PAD * 4);
       for (int idx = threadIdx.x; idx < ACT_ROWS * p.r; idx += ACT_THREADS) {
         const int row = idx / p.r, col = idx % p.r;
-        const int grow = row0 + row;
-        if (grow >= p.M) continue;
         float v = 0.0f;
 #pragma unroll
         for (int w = 0; w < ACT_WARPS; ++w) v += red[(w * ACT_ROWS + row) * R_PAD + col];
-        p.D[static_cast<size_t>(grow) * p.r + col] = static_cast<uint16_t>(pack_bf16x2(-v, 0.0f) & 0xFFFFu);
+        st_shared_cluster_f32(dst0 + static_cast<uint32_t>(row * R_PAD + col) * 4u, v);
+      }
+      __syncwarp();
+      cluster_sync_all();
+      if (kpart == 0 && !*abort_flag) {
+        for (int idx = threadIdx.x; idx < ACT_ROWS * p.r; idx += ACT_THREADS) {
+          const int row = idx / p.r, col = idx % p.r;
+          const int grow = row0 + row;
+          if (grow >= p.M) continue;
+          float v = 0.0f;
+          for (int c = 0; c < p.ks; ++c) v += recv[(c * ACT_ROWS + row) * R_PAD + col];
+          p.D[static_cast<size_t>(grow) * p.r + col] = static_cast<uint16_t>(pack_bf16x2(-v, 0.0f) & 0xFFFFu);
+        }
       }
     }
   }

@@ -153,10 +153,44 @@ svdq_status launch_act(const CUtensorMap& tx, const ActParams& p, cudaStream_t s
                                     smem);
   });
   if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(act)");
-  const int grid = p.M_pad / ACT_ROWS;
-  act_quant_kernel<R_PAD><<<grid, ACT_THREADS, smem, st>>>(tx, p);
+  const int grid = p.M_pad / ACT_ROWS * p.ks;
+  if (p.ks == 1) {
+    act_quant_kernel<R_PAD><<<grid, ACT_THREADS, smem, st>>>(tx, p);
+  } else {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(ACT_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(p.ks);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, act_quant_kernel<R_PAD>, tx, p);
+    if (e != cudaSuccess) return cuda_fail(e, "act_quant_kernel (cluster) launch");
+  }
   SVDQ_CHECK_LAUNCH("act_quant_kernel");
   return SVDQ_OK;
+}
+
+// K split of the activation kernel: with few row blocks of 16 (small M), a
+// cluster of ks CTAs shares each block so that more SMs stream X.  The largest
+// ks <= 8 with K % (64 ks) == 0, at least one 64-column sub-tile per warp
+// (K / ks >= 512) and at most one CTA per SM.  SVDQ_ACT_KS=ks overrides it
+// when K % (64 ks) == 0.
+int act_k_split(int M, int K) {
+  if (const char* e = std::getenv("SVDQ_ACT_KS")) {
+    const int v = std::atoi(e);
+    if (v >= 1 && v <= ACT_MAX_KS && K % (ACT_SUB * v) == 0) return v;
+  }
+  const int blocks = (M + ACT_ROWS - 1) / ACT_ROWS;
+  int ks = 1;
+  for (int c = 2; c <= ACT_MAX_KS; ++c)
+    if (K % (ACT_SUB * c) == 0 && K / c >= ACT_SUB * ACT_WARPS && blocks * c <= num_sms()) ks = c;
+  return ks;
 }
 
 template <int BN, int R_PAD>
@@ -207,6 +241,7 @@ svdq_status quantize_act_impl(const uint16_t* X, int M, const svdq_weight* w, ui
   p.K = K;
   p.r = r;
   p.M_pad = m_pad_of(M);
+  p.ks = act_k_split(M, K);
   switch (rp) {
     case 0: return launch_act<0>(tx, p, st);
     case 16: return launch_act<16>(tx, p, st);
