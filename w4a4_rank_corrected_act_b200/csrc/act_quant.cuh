@@ -105,6 +105,9 @@ __global__ void __launch_bounds__(ACT_THREADS, 2)
   }
   for (int c = threadIdx.x; c < 128; c += ACT_THREADS) tab[c] = e4m3_table_entry(c);
   __syncthreads();   // barriers, the E4M3 table and the abort flag are initialised
+  // the GEMM that consumes this kernel's output may be launched now: it loads
+  // weights until its griddepcontrol.wait, which waits for this grid to finish
+  pdl_launch_dependents();
 
   const int my_count = nsub > warp ? (nsub - warp + ACT_WARPS - 1) / ACT_WARPS : 0;
   auto issue = [&](int jj) {

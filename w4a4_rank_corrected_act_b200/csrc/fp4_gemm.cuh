@@ -264,6 +264,42 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       for (int s = 0; s < S; ++s) fill_parity[s] = -1;
       const uint32_t tx_main = GEMM_A_TILE + Cfg::kBTile + GEMM_SFA_TILE + Cfg::kSFBTile;
       const uint32_t tx_lr = (GEMM_BM + BN) * R_PAD * 2;
+      // Programmatic dependent launch: this grid may start while the kernel
+      // that writes the activation codes, scales and D is still running.  The
+      // weight halves of the first S stages are loaded at once; their
+      // activation halves wait for that kernel (griddepcontrol.wait), as does
+      // everything after them.  The stage barriers count both halves' bytes.
+      struct Deferred {
+        int stage, kb, m0, mb;   // kb < 0: the low-rank slot (D tile)
+      };
+      Deferred deferred[S];
+      int ndeferred = 0;
+      bool dependency_met = false;
+      auto load_activation = [&](const Deferred& q) {
+        if (q.kb < 0) {
+          tma_load_2d(stage_a(q.stage), &tm_d, full_bar(q.stage), 0, q.m0);
+        } else {
+          tma_load_2d(stage_a(q.stage), &tm_a, full_bar(q.stage), q.kb * 128, q.m0);
+          bulk_load(stage_sfa(q.stage), p.x_scales + (static_cast<size_t>(q.mb) * k_tiles64 + q.kb * 4) * 512,
+                    GEMM_SFA_TILE, full_bar(q.stage));
+        }
+      };
+      auto meet_dependency = [&]() {
+        pdl_wait();
+        for (int i = 0; i < ndeferred; ++i) load_activation(deferred[i]);
+        ndeferred = 0;
+        dependency_met = true;
+      };
+      // issue the activation half of a stage now, or defer it (first S stages)
+      auto activation_half = [&](int st, int kb, int m0, int mb) {
+        const Deferred q{st, kb, m0, mb};
+        if (dependency_met) {
+          load_activation(q);
+        } else {
+          deferred[ndeferred++] = q;
+          if (ndeferred == S) meet_dependency();   // the ring is full: nothing more to overlap
+        }
+      };
       bool ok = true;
       for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
         const int mb = t % p.m_tiles, nb = t / p.m_tiles;
@@ -271,28 +307,27 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         if (R_PAD > 0) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1, abort_flag, KID_GEMM, 1)) { ok = false; break; }
           mbar_arrive_expect_tx(full_bar(stage), tx_lr);
-          tma_load_2d(stage_a(stage), &tm_d, full_bar(stage), 0, m0);
           tma_load_2d(stage_b(stage), &tm_l2, full_bar(stage), 0, n0);
+          activation_half(stage, -1, m0, mb);
           fill_parity[stage] = static_cast<int8_t>(phase);
           if (++stage == S) { stage = 0; phase ^= 1; }
         }
         for (int kb = 0; kb < kb_per_tile; ++kb) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1, abort_flag, KID_GEMM, 2)) { ok = false; break; }
           mbar_arrive_expect_tx(full_bar(stage), tx_main);
-          tma_load_2d(stage_a(stage), &tm_a, full_bar(stage), kb * 128, m0);
           tma_load_2d(stage_b(stage), &tm_b, full_bar(stage), kb * 128, n0);
-          bulk_load(stage_sfa(stage),
-                    p.x_scales + (static_cast<size_t>(mb) * k_tiles64 + kb * 4) * 512,
-                    GEMM_SFA_TILE, full_bar(stage));
 #pragma unroll
           for (int g = 0; g < BN / 128; ++g)
             bulk_load(stage_sfb(stage) + g * GEMM_SFA_TILE,
                       p.w_scales + (static_cast<size_t>(n0 / 128 + g) * k_tiles64 + kb * 4) * 512,
                       GEMM_SFA_TILE, full_bar(stage));
+          activation_half(stage, kb, m0, mb);
           fill_parity[stage] = static_cast<int8_t>(phase);
           if (++stage == S) { stage = 0; phase ^= 1; }
         }
       }
+      // fewer than S stages in all, or an abort: complete the deferred stages
+      if (!dependency_met) meet_dependency();
       if (*abort_flag) {
         for (int s = 0; s < S; ++s)
           if (fill_parity[s] >= 0) mbar_wait_drain(full_bar(s), static_cast<uint32_t>(fill_parity[s]));

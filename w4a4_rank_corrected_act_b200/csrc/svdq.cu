@@ -206,7 +206,21 @@ svdq_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUte
   });
   if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(gemm)");
   const int grid = std::min(p.num_tiles, num_sms());
-  fp4_gemm_kernel<BN, R_PAD><<<grid, GEMM_THREADS, Cfg::kSmemBytes, st>>>(ta, tb, td, tl2, ty, p);
+  // programmatic dependent launch: the kernel may start while the preceding
+  // kernel of the stream (the activation kernel) finishes; it waits for it
+  // before reading anything that kernel writes
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(GEMM_THREADS);
+  cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, fp4_gemm_kernel<BN, R_PAD>, ta, tb, td, tl2, ty, p);
+  if (e != cudaSuccess) return cuda_fail(e, "fp4_gemm_kernel launch");
   SVDQ_CHECK_LAUNCH("fp4_gemm_kernel");
   return SVDQ_OK;
 }
