@@ -326,6 +326,8 @@ def run_native(args):
             "pct_fp4_peak": {"of_spec_9000": round(value / FP4_SPEC_TFLOPS, 4),
                              "of_measured_bf16x4": round(value / fp4_peak, 4)},
             "us_per_layer": round(ms_per_step * 1e3, 2),
+            "step_us_percentiles": {"p50": round(float(np.percentile(step_ms, 50)) * 1e3, 2),
+                                    "p95": round(float(np.percentile(step_ms, 95)) * 1e3, 2)},
             "roofline": roofline,
             "kernels": {"act_quant": act},
             "e2e": e2e,
@@ -374,9 +376,29 @@ def cpu_baseline(spec, d, exp, budget_s=15.0, rows=256):
         if el >= budget_s or n >= 50:
             break
     flops = 2.0 * rows * spec.N * spec.K * n
-    return {"value": flops / el / 1e12, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
-            "sample": f"{rows} of {spec.M} token rows x {n} repetitions ({el:.1f} s), full K and N; "
-                      "oracle forward incl. per-call weight dequantisation"}
+    out = {"value": flops / el / 1e12, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+           "sample": f"{rows} of {spec.M} token rows x {n} repetitions ({el:.1f} s), full K and N; "
+                     "oracle forward incl. per-call weight dequantisation"}
+    # the same forward by stage (all cores), and on one BLAS thread (a smaller sample)
+    Xs = X[:64]
+    t0 = time.perf_counter()
+    act = ref.quantize_act(Xs, prep["inv_lambda"], prep["L1"])
+    t1 = time.perf_counter()
+    ref.dequantize(act["x_codes"], act["x_scales"]) @ ref.dequantize(prep["w_codes"], prep["w_scales"]).T
+    t2 = time.perf_counter()
+    out["stages_s_64_rows"] = {"quantise_x": round(t1 - t0, 4), "dequantise_and_gemm": round(t2 - t1, 4)}
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            t0 = time.perf_counter()
+            ref.linear_forward(Xs, prep)
+            el1 = time.perf_counter() - t0
+        out["value_1_thread"] = 2.0 * 64 * spec.N * spec.K / el1 / 1e12
+        out["sample_1_thread"] = "64 token rows, one forward"
+    except Exception as e:  # threadpoolctl missing or BLAS not controllable
+        out["value_1_thread"] = None
+        out["sample_1_thread"] = f"not measured ({type(e).__name__})"
+    return out
 
 
 def run_reference(args):

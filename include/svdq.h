@@ -270,6 +270,16 @@ svdq_status svdq_selftest_wait_timeout(uint64_t limit_ns, void* stream);
  * of 3.  The paper has no counterpart: this is test support. */
 svdq_status svdq_selftest_quotient(uint64_t* counts);
 
+/* Numerics self-test of the hardware conversions the kernels round with, on
+ * the current device (synchronous).  For every non-negative finite float32 x
+ * it compares cvt.rn.satfinite.e4m3x2 with the nearest of the 127 finite E4M3
+ * values (ties to the even code, saturating at 448), cvt.rn.satfinite.e2m1x2
+ * with the E2M1 thresholds 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5 (ties to even),
+ * and cvt.rn.bf16x2 with round-to-nearest-even on the upper 16 bits, and
+ * writes the mismatch counts to counts[0..2] (host array of 3; all 0 on a
+ * correct device).  The paper has no counterpart: this is test support. */
+svdq_status svdq_selftest_conversions(uint64_t* counts);
+
 #ifdef __cplusplus
 }  /* extern "C" */
 #endif

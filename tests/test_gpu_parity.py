@@ -365,6 +365,14 @@ def test_quantiser_quotient_exhaustive():
     assert (q_bad, c_bad) == (0, 0), (q_bad, c_bad, q_sub)
 
 
+def test_device_conversions_exhaustive():
+    """The hardware E4M3, E2M1 and bf16 conversions the kernels round with agree
+    with the formats' definitions on every non-negative finite float32 (the
+    oracle's table-driven conversions are pinned to the same definitions by
+    the CPU tests)."""
+    assert svdq.svdq_selftest_conversions() == (0, 0, 0)
+
+
 def test_device_status_clean():
     torch().cuda.synchronize()
     assert svdq.svdq_get_device_status(stream()) == 0

@@ -64,6 +64,7 @@ SIGNATURES = {
     "svdq_clear_device_status": (_I, [_P]),
     "svdq_selftest_wait_timeout": (_I, [ctypes.c_uint64, _P]),
     "svdq_selftest_quotient": (_I, [ctypes.POINTER(ctypes.c_uint64)]),
+    "svdq_selftest_conversions": (_I, [ctypes.POINTER(ctypes.c_uint64)]),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -215,6 +216,14 @@ def svdq_selftest_quotient() -> tuple:
     its exhaustive sweep; the first two are 0 on a correct build."""
     out = (ctypes.c_uint64 * 3)()
     _call("svdq_selftest_quotient", out)
+    return int(out[0]), int(out[1]), int(out[2])
+
+
+def svdq_selftest_conversions() -> tuple:
+    """(E4M3, E2M1, bf16) mismatch counts of the device conversions over every
+    non-negative finite float32; all 0 on a correct device."""
+    out = (ctypes.c_uint64 * 3)()
+    _call("svdq_selftest_conversions", out)
     return int(out[0]), int(out[1]), int(out[2])
 
 

@@ -560,6 +560,51 @@ __global__ void selftest_quotient_kernel() {
   }
 }
 
+// Exhaustive check of the hardware conversions the kernels round with, for
+// every non-negative finite float32 x, against the formats' definitions:
+// counts[0] E4M3 (cvt.rn.satfinite.e4m3x2: nearest of the 127 finite E4M3
+// values, ties to the even code, saturating at 448), counts[1] E2M1
+// (cvt.rn.satfinite.e2m1x2, thresholds as above), counts[2] bf16
+// (cvt.rn.bf16x2: round to nearest even on the upper 16 bits).
+__device__ unsigned long long g_conversion_mismatch[3];
+
+__global__ void selftest_conversion_kernel() {
+  __shared__ float e4m3[127];
+  for (int c = threadIdx.x; c < 127; c += blockDim.x) e4m3[c] = e4m3_to_f32(static_cast<uint32_t>(c));
+  __syncthreads();
+  const float thr[7] = {0.25f, 0.75f, 1.25f, 1.75f, 2.5f, 3.5f, 5.0f};
+  unsigned long long bad[3] = {0ull, 0ull, 0ull};
+  for (uint32_t u = blockIdx.x * blockDim.x + threadIdx.x; u < 0x7F800000u; u += gridDim.x * blockDim.x) {
+    const float x = __uint_as_float(u);
+    // E4M3: largest code whose value is <= x, then the nearer neighbour
+    uint32_t want;
+    if (x >= 448.0f) {
+      want = 126u;
+    } else {
+      int lo = 0, hi = 126;   // e4m3[lo] <= x < e4m3[hi]
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (e4m3[mid] <= x) lo = mid; else hi = mid;
+      }
+      const float dl = x - e4m3[lo], dh = e4m3[hi] - x;   // exact: both within a binade of x
+      want = static_cast<uint32_t>(dl < dh ? lo : dh < dl ? hi : ((lo & 1) ? hi : lo));
+    }
+    if (e4m3_rn_satfinite(x) != want) ++bad[0];
+    // E2M1
+    uint32_t w2 = 0;
+#pragma unroll
+    for (int k = 0; k < 7; ++k)
+      if (x > thr[k] || (x == thr[k] && (k & 1))) w2 = static_cast<uint32_t>(k + 1);
+    const float a[8] = {x, x, x, x, x, x, x, x};
+    if ((e2m1x8_magnitudes(a) & 15u) != w2) ++bad[1];
+    // bf16
+    const uint32_t wb = (u + 0x7FFFu + ((u >> 16) & 1u)) >> 16;
+    if ((pack_bf16x2(x, 0.0f) & 0xFFFFu) != wb) ++bad[2];
+  }
+  for (int i = 0; i < 3; ++i)
+    if (bad[i]) atomicAdd(&g_conversion_mismatch[i], bad[i]);
+}
+
 // --------------------------------------------------------------------------
 // Fixed device scratch for svdq_linear_forward_noalloc.  Every GPU that loads
 // this library holds it until the process exits.  Host code only ever sees a
@@ -891,6 +936,19 @@ svdq_status svdq_selftest_quotient(uint64_t* counts) {
   SVDQ_CUDA(cudaDeviceSynchronize());
   unsigned long long out[3];
   SVDQ_CUDA(cudaMemcpyFromSymbol(out, g_quotient_mismatch, sizeof(out)));
+  for (int i = 0; i < 3; ++i) counts[i] = out[i];
+  return SVDQ_OK;
+}
+
+svdq_status svdq_selftest_conversions(uint64_t* counts) {
+  if (counts == nullptr) return SVDQ_ERR_INVALID_ARG;
+  const unsigned long long z[3] = {0ull, 0ull, 0ull};
+  SVDQ_CUDA(cudaMemcpyToSymbol(g_conversion_mismatch, z, sizeof(z)));
+  selftest_conversion_kernel<<<num_sms() * 8, 256>>>();
+  SVDQ_CHECK_LAUNCH("selftest_conversion_kernel");
+  SVDQ_CUDA(cudaDeviceSynchronize());
+  unsigned long long out[3];
+  SVDQ_CUDA(cudaMemcpyFromSymbol(out, g_conversion_mismatch, sizeof(out)));
   for (int i = 0; i < 3; ++i) counts[i] = out[i];
   return SVDQ_OK;
 }
