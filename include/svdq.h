@@ -232,6 +232,35 @@ svdq_status svdq_weight_export(const svdq_weight* w, uint8_t* host_codes, uint8_
                                uint16_t* host_L1, uint16_t* host_L2t, float* host_inv_lambda,
                                void* stream);
 
+/* Checkpoint import, the inverse of svdq_weight_export: fill a bound weight
+ * from host buffers in the same logical layouts (codes N x K/2, scales
+ * N x K/16 row-major, L1 K x r, L2t N x r, inv_lambda K) plus the bias (N
+ * bf16; required exactly when w->has_bias).  The scales are converted to the
+ * tile layout on the host and L1t is regenerated from L1 on the device.  The
+ * watch-ia.com page's offline loop ("quantise, package, load and verify")
+ * needs this load step.  Synchronises `stream`.  SVDQ_ERR_INVALID_ARG for a
+ * missing buffer. */
+svdq_status svdq_weight_import(const svdq_weight* w, const uint8_t* host_codes, const uint8_t* host_scales,
+                               const uint16_t* host_L1, const uint16_t* host_L2t,
+                               const float* host_inv_lambda, const uint16_t* host_bias, void* stream);
+
+/* Calibration statistics (offline): colmax[k] = max(colmax[k], max_m |A[m][k]|)
+ * for a device rows x K bf16 matrix A, row-major.  colmax is a device float
+ * array of K entries; zero it before the first batch, then call once per
+ * calibration batch of activations.  Asynchronous on `stream`. */
+svdq_status svdq_calib_absmax(const uint16_t* A, int rows, int K, float* colmax, void* stream);
+
+/* Smoothing factors from calibration statistics (offline):
+ *   lambda[k] = f32( x_k^alpha / w_k^(1 - alpha) ),  x_k = x_absmax[k],
+ *   w_k = max_n |W[n][k]|, evaluated in float64; alpha = 0.5 is evaluated as
+ *   f32(sqrt(x_k / w_k)); lambda[k] = 1 where x_k or w_k is 0.
+ * alpha in [0, 1] is the migration strength: the share of each input
+ * channel's activation range moved into the weight (0.5 balances the two
+ * maxima).  W device N x K bf16; x_absmax and lambda device, K floats.
+ * Asynchronous on `stream`; lambda is then the input of svdq_prepare_weight. */
+svdq_status svdq_calibrate_lambda(const float* x_absmax, const uint16_t* W, int N, int K, float alpha,
+                                  float* lambda, void* stream);
+
 /* Host-only layout conversions between logical [rows][K/16] scales and the
  * tile layout (rows of the tile layout are `rows` rounded up to 128; padding
  * entries are written as 0 by to_native and ignored by to_logical). */

@@ -234,6 +234,33 @@ def dequantize(packed: np.ndarray, scales: np.ndarray) -> np.ndarray:
 # ---------------------------------------------------------------------------
 
 
+def column_absmax(a_bits: np.ndarray) -> np.ndarray:
+    """max over rows of |A[:, k]| for a bf16 matrix (float32; exact)."""
+    return np.abs(bf16_to_f64(a_bits)).max(axis=0).astype(np.float32)
+
+
+def calibrate_lambda(x_absmax: np.ndarray, w_bits: np.ndarray, alpha: float = 0.5) -> np.ndarray:
+    """Smoothing factors from calibration statistics (offline step).
+
+    The pages move each input channel's activation outliers into the weight
+    (chaosnode.de "Nunchaku Lite ...", section "Die Technik: SVDQuant") and
+    calibrate offline (watch-ia.com, last paragraphs), but give no formula.
+    Reading: lambda_k = x_k^alpha / w_k^(1-alpha) with x_k = max|X[:, k]| over
+    the calibration activations, w_k = max|W[:, k]|, in float64, rounded once to
+    float32; alpha = 0.5 (the inputs' recipe) is evaluated as sqrt(x_k / w_k);
+    lambda_k = 1 where either maximum is 0.
+    """
+    x = np.asarray(x_absmax, dtype=np.float64)
+    w = column_absmax(w_bits).astype(np.float64)
+    lam = np.ones_like(x)
+    ok = (x > 0) & (w > 0)
+    if alpha == 0.5:
+        lam[ok] = np.sqrt(x[ok] / w[ok])
+    else:
+        lam[ok] = np.power(x[ok], alpha) / np.power(w[ok], 1.0 - alpha)
+    return lam.astype(np.float32)
+
+
 def inv_lambda_of(lam: np.ndarray) -> np.ndarray:
     lam = np.asarray(lam, dtype=np.float32)
     return (np.float32(1.0) / lam).astype(np.float32)

@@ -58,6 +58,9 @@ SIGNATURES = {
     "svdq_linear_forward_host": (_I, [_P, _I, _WP, _P, _P, _P, _P, _SZ, _P]),
     "svdq_linear_forward_noalloc": (_I, [_P, _I, _WP, _P, _P]),
     "svdq_weight_export": (_I, [_WP, _P, _P, _P, _P, _P, _P]),
+    "svdq_weight_import": (_I, [_WP, _P, _P, _P, _P, _P, _P, _P]),
+    "svdq_calib_absmax": (_I, [_P, _I, _I, _P, _P]),
+    "svdq_calibrate_lambda": (_I, [_P, _P, _I, _I, ctypes.c_float, _P, _P]),
     "svdq_scales_to_logical": (_I, [_P, _I, _I, _P]),
     "svdq_scales_to_native": (_I, [_P, _I, _I, _P]),
     "svdq_get_device_status": (_I, [_P, ctypes.POINTER(ctypes.c_uint32)]),
@@ -185,6 +188,21 @@ def svdq_weight_export(w: svdq_weight, host_codes: int, host_scales: int, host_L
           host_L1 or None, host_L2t or None, host_inv_lambda or None, stream or None)
 
 
+def svdq_weight_import(w: svdq_weight, host_codes: int, host_scales: int, host_L1: int,
+                       host_L2t: int, host_inv_lambda: int, host_bias: int, stream: int) -> None:
+    _call("svdq_weight_import", ctypes.byref(w), host_codes, host_scales, host_L1 or None,
+          host_L2t or None, host_inv_lambda, host_bias or None, stream or None)
+
+
+def svdq_calib_absmax(A: int, rows: int, K: int, colmax: int, stream: int) -> None:
+    _call("svdq_calib_absmax", A, rows, K, colmax, stream or None)
+
+
+def svdq_calibrate_lambda(x_absmax: int, W: int, N: int, K: int, alpha: float, lam: int,
+                          stream: int) -> None:
+    _call("svdq_calibrate_lambda", x_absmax, W, N, K, float(alpha), lam, stream or None)
+
+
 def svdq_scales_to_logical(native: int, rows: int, K: int, logical: int) -> None:
     _call("svdq_scales_to_logical", native, rows, K, logical)
 
@@ -248,14 +266,7 @@ class SvdqLinear:
     def __init__(self, W, lam, bias=None, r: int = 32, stream=None):
         import torch
         N, K = W.shape
-        self.N, self.K, self.r = int(N), int(K), int(r)
-        self.has_bias = bias is not None
-        nbytes = svdq_weight_bytes(self.N, self.K, self.r, int(self.has_bias))
-        if nbytes == 0:
-            raise SvdqError("svdq_weight_bytes", 2, f"N={N} K={K} r={r}")
-        self.buf = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
-        self.w = svdq_weight_bind(self.buf.data_ptr(), nbytes, self.N, self.K, self.r,
-                                  int(self.has_bias))
+        self._bind(int(N), int(K), int(r), bias is not None, W.device)
         ws_bytes = svdq_prepare_workspace_bytes(self.N, self.K, self.r)
         ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=W.device)
         Wc = W.contiguous()
@@ -265,6 +276,63 @@ class SvdqLinear:
                             self.w, ws.data_ptr(), ws_bytes, _stream_handle(stream))
         torch.cuda.current_stream().synchronize() if stream is None else stream.synchronize()
         del ws
+
+    def _bind(self, N: int, K: int, r: int, has_bias: bool, device) -> None:
+        import torch
+        self.N, self.K, self.r = N, K, r
+        self.has_bias = has_bias
+        nbytes = svdq_weight_bytes(self.N, self.K, self.r, int(self.has_bias))
+        if nbytes == 0:
+            raise SvdqError("svdq_weight_bytes", 2, f"N={N} K={K} r={r}")
+        self.buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.w = svdq_weight_bind(self.buf.data_ptr(), nbytes, self.N, self.K, self.r,
+                                  int(self.has_bias))
+
+    @classmethod
+    def from_export(cls, exp: dict, bias=None, device="cuda", stream=None):
+        """A layer from host arrays in the layouts of ``export()`` (bias: N uint16
+        bf16 bits or None), loaded with ``svdq_weight_import``."""
+        import numpy as np
+        self = cls.__new__(cls)
+        N, K2 = exp["w_codes"].shape
+        r = int(exp["L1"].shape[1]) if exp.get("L1") is not None else 0
+        self._bind(int(N), int(K2) * 2, r, bias is not None, device)
+        # every host array stays referenced until the (synchronous) import returns
+        codes = np.ascontiguousarray(exp["w_codes"], dtype=np.uint8)
+        scales = np.ascontiguousarray(exp["w_scales"], dtype=np.uint8)
+        L1 = np.ascontiguousarray(exp["L1"], dtype=np.uint16) if r else None
+        L2t = np.ascontiguousarray(exp["L2t"], dtype=np.uint16) if r else None
+        inv = np.ascontiguousarray(exp["inv_lambda"], dtype=np.float32)
+        b = np.ascontiguousarray(bias, dtype=np.uint16) if bias is not None else None
+        svdq_weight_import(self.w, codes.ctypes.data, scales.ctypes.data,
+                           L1.ctypes.data if r else 0, L2t.ctypes.data if r else 0, inv.ctypes.data,
+                           b.ctypes.data if b is not None else 0, _stream_handle(stream))
+        return self
+
+    def bias_host(self):
+        """The layer's bias as uint16 bf16 bits (numpy), or None."""
+        if not self.has_bias:
+            return None
+        off = self.w.bias - self.buf.data_ptr()
+        return self.buf[off:off + 2 * self.N].cpu().numpy().view("uint16").copy()
+
+    def save(self, path) -> None:
+        """Write the prepared weight (logical layouts, bias included) to an .npz file."""
+        import numpy as np
+        exp = self.export()
+        extra = {"bias": self.bias_host()} if self.has_bias else {}
+        np.savez(path, format=np.array("svdq-w4a4-nvfp4-1"), N=self.N, K=self.K, r=self.r, **exp, **extra)
+
+    @classmethod
+    def load(cls, path, device="cuda", stream=None):
+        """A layer from a file written by ``save``."""
+        import numpy as np
+        with np.load(path) as z:
+            if str(z["format"]) != "svdq-w4a4-nvfp4-1":
+                raise ValueError(f"{path}: not an SVDQuant weight file")
+            exp = {k: z[k] for k in ("w_codes", "w_scales", "L1", "L2t", "inv_lambda")}
+            bias = z["bias"] if "bias" in z.files else None
+        return cls.from_export(exp, bias=bias, device=device, stream=stream)
 
     def workspace_bytes(self, M: int) -> int:
         return svdq_forward_workspace_bytes(M, self.N, self.K, self.r)
@@ -293,3 +361,22 @@ class SvdqLinear:
                            L1.ctypes.data if self.r else 0, L2t.ctypes.data if self.r else 0,
                            inv.ctypes.data, _stream_handle())
         return dict(w_codes=codes, w_scales=scales, L1=L1, L2t=L2t, inv_lambda=inv)
+
+
+def calibrate_lambda(W, X_batches, alpha: float = 0.5, stream=None):
+    """Smoothing factors for the weight W (N x K bf16, device) from calibration
+    activations (an iterable of M_i x K bf16 device tensors): the column
+    maxima of |X| over all batches (svdq_calib_absmax), then
+    svdq_calibrate_lambda with migration strength alpha.  Returns a device
+    float32 tensor of K entries, the ``lam`` input of SvdqLinear."""
+    import torch
+    N, K = W.shape
+    sh = _stream_handle(stream)
+    colmax = torch.zeros(K, dtype=torch.float32, device=W.device)
+    for X in X_batches:
+        Xc = X.contiguous()
+        svdq_calib_absmax(Xc.data_ptr(), int(Xc.shape[0]), int(K), colmax.data_ptr(), sh)
+    lam = torch.empty(K, dtype=torch.float32, device=W.device)
+    Wc = W.contiguous()
+    svdq_calibrate_lambda(colmax.data_ptr(), Wc.data_ptr(), int(N), int(K), alpha, lam.data_ptr(), sh)
+    return lam

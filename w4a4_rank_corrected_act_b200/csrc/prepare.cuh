@@ -263,4 +263,42 @@ __global__ void __launch_bounds__(256) prep_residual_kernel(const float* __restr
   }
 }
 
+// ---------------------------------------------------------------------------
+// Calibration statistics: colmax[k] = max(colmax[k], max_m |A[m][k]|) for a
+// row-major rows x K bf16 matrix (activations X, or the weight W).  Thread t
+// of the grid owns column pair 2 (t % (K/2)) and a strided slice of the rows;
+// the running maximum is kept as float bits, whose integer order matches the
+// order of non-negative floats.
+__global__ void calib_absmax_kernel(const uint16_t* __restrict__ A, int rows, int K,
+                                    unsigned int* __restrict__ colmax_bits) {
+  const long long pairs = K / 2;
+  const long long T = static_cast<long long>(gridDim.x) * blockDim.x;
+  const long long slices = T / pairs > 0 ? T / pairs : 1;
+  for (long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; idx < pairs * slices;
+       idx += T) {
+    const long long c = idx % pairs, slice = idx / pairs;
+    unsigned int m0 = 0u, m1 = 0u;
+    for (long long row = slice; row < rows; row += slices) {
+      const uint32_t v = *reinterpret_cast<const uint32_t*>(A + row * K + 2 * c);
+      m0 = max(m0, (v & 0x7FFFu) << 16);   // |bf16| as float32 bits
+      m1 = max(m1, v & 0x7FFF0000u);
+    }
+    if (m0) atomicMax(colmax_bits + 2 * c, m0);
+    if (m1) atomicMax(colmax_bits + 2 * c + 1, m1);
+  }
+}
+
+// lambda[k] = f32(x^alpha / w^(1 - alpha)) in float64 from the activation and
+// weight column maxima (w_in_lambda holds max|W[:, k]| on entry); alpha = 0.5
+// is evaluated as f32(sqrt(x / w)); 1 where either maximum is 0.
+__global__ void calib_lambda_kernel(const float* __restrict__ x_absmax, int K, double alpha,
+                                    float* __restrict__ lambda) {
+  for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < K; k += gridDim.x * blockDim.x) {
+    const double x = x_absmax[k], w = lambda[k];
+    double l = 1.0;
+    if (x > 0.0 && w > 0.0) l = alpha == 0.5 ? sqrt(x / w) : pow(x, alpha) / pow(w, 1.0 - alpha);
+    lambda[k] = static_cast<float>(l);
+  }
+}
+
 }  // namespace svdq

@@ -476,6 +476,13 @@ int syevd_lwork(int n, cusolverDnHandle_t h) {
   return lwork;
 }
 
+void to_native(const uint8_t* logical, int rows, int K, uint8_t* native) {
+  const int kb = K / 16;
+  std::memset(native, 0, static_cast<size_t>(m_pad_of(rows)) * kb);
+  for (int i = 0; i < rows; ++i)
+    for (int j = 0; j < kb; ++j) native[sf_offset(i, j, K)] = logical[static_cast<size_t>(i) * kb + j];
+}
+
 void to_logical(const uint8_t* native, int rows, int K, uint8_t* logical) {
   const int kb = K / 16;
   for (int i = 0; i < rows; ++i)
@@ -895,6 +902,59 @@ svdq_status svdq_weight_export(const svdq_weight* w, uint8_t* host_codes, uint8_
   return SVDQ_OK;
 }
 
+svdq_status svdq_weight_import(const svdq_weight* w, const uint8_t* host_codes, const uint8_t* host_scales,
+                               const uint16_t* host_L1, const uint16_t* host_L2t,
+                               const float* host_inv_lambda, const uint16_t* host_bias, void* stream) {
+  svdq_status s = check_weight(w);
+  if (s != SVDQ_OK) return s;
+  if (host_codes == nullptr || host_scales == nullptr || host_inv_lambda == nullptr ||
+      (w->r > 0 && (host_L1 == nullptr || host_L2t == nullptr)) || (w->has_bias != 0) != (host_bias != nullptr))
+    return SVDQ_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t N = w->N, K = w->K, r = w->r;
+  std::vector<uint8_t> native(N * K / 16);
+  to_native(host_scales, w->N, w->K, native.data());
+  SVDQ_CUDA(cudaMemcpyAsync(w->w_codes, host_codes, N * K / 2, cudaMemcpyHostToDevice, st));
+  SVDQ_CUDA(cudaMemcpyAsync(w->w_scales, native.data(), native.size(), cudaMemcpyHostToDevice, st));
+  if (r) {
+    SVDQ_CUDA(cudaMemcpyAsync(w->L1, host_L1, K * r * 2, cudaMemcpyHostToDevice, st));
+    SVDQ_CUDA(cudaMemcpyAsync(w->L2t, host_L2t, N * r * 2, cudaMemcpyHostToDevice, st));
+    l1_fragment_kernel<<<num_sms() * 2, 256, 0, st>>>(w->L1, w->K, w->r, w->L1f);
+    SVDQ_CHECK_LAUNCH("l1_fragment_kernel");
+  }
+  SVDQ_CUDA(cudaMemcpyAsync(w->inv_lambda, host_inv_lambda, K * 4, cudaMemcpyHostToDevice, st));
+  if (host_bias) SVDQ_CUDA(cudaMemcpyAsync(w->bias, host_bias, N * 2, cudaMemcpyHostToDevice, st));
+  // the staging copy of the scales must outlive its transfer
+  SVDQ_CUDA(cudaStreamSynchronize(st));
+  return SVDQ_OK;
+}
+
+svdq_status svdq_calib_absmax(const uint16_t* A, int rows, int K, float* colmax, void* stream) {
+  if (A == nullptr || colmax == nullptr || rows < 0 || K <= 0 || K % 2) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(colmax)) return SVDQ_ERR_MISALIGNED;
+  if (rows == 0) return SVDQ_OK;
+  calib_absmax_kernel<<<num_sms() * 4, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      A, rows, K, reinterpret_cast<unsigned int*>(colmax));
+  SVDQ_CHECK_LAUNCH("calib_absmax_kernel");
+  return SVDQ_OK;
+}
+
+svdq_status svdq_calibrate_lambda(const float* x_absmax, const uint16_t* W, int N, int K, float alpha,
+                                  float* lambda, void* stream) {
+  if (x_absmax == nullptr || W == nullptr || lambda == nullptr || N <= 0 || K <= 0 || K % 2 ||
+      !(alpha >= 0.0f && alpha <= 1.0f))
+    return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(x_absmax) || !aligned16(W) || !aligned16(lambda)) return SVDQ_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // max|W[:, k]| is gathered in lambda itself, then turned into lambda in place
+  SVDQ_CUDA(cudaMemsetAsync(lambda, 0, static_cast<size_t>(K) * 4, st));
+  calib_absmax_kernel<<<num_sms() * 4, 256, 0, st>>>(W, N, K, reinterpret_cast<unsigned int*>(lambda));
+  SVDQ_CHECK_LAUNCH("calib_absmax_kernel");
+  calib_lambda_kernel<<<(K + 255) / 256, 256, 0, st>>>(x_absmax, K, static_cast<double>(alpha), lambda);
+  SVDQ_CHECK_LAUNCH("calib_lambda_kernel");
+  return SVDQ_OK;
+}
+
 svdq_status svdq_scales_to_logical(const uint8_t* native, int rows, int K, uint8_t* logical) {
   if (native == nullptr || logical == nullptr || rows < 0 || K <= 0 || K % 64) return SVDQ_ERR_INVALID_ARG;
   to_logical(native, rows, K, logical);
@@ -903,10 +963,7 @@ svdq_status svdq_scales_to_logical(const uint8_t* native, int rows, int K, uint8
 
 svdq_status svdq_scales_to_native(const uint8_t* logical, int rows, int K, uint8_t* native) {
   if (native == nullptr || logical == nullptr || rows < 0 || K <= 0 || K % 64) return SVDQ_ERR_INVALID_ARG;
-  const int kb = K / 16;
-  std::memset(native, 0, static_cast<size_t>(m_pad_of(rows)) * kb);
-  for (int i = 0; i < rows; ++i)
-    for (int j = 0; j < kb; ++j) native[sf_offset(i, j, K)] = logical[static_cast<size_t>(i) * kb + j];
+  to_native(logical, rows, K, native);
   return SVDQ_OK;
 }
 
