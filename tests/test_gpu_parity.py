@@ -242,7 +242,8 @@ def test_gemm_parity(M, K, N, r, pair, monkeypatch):
     o = ref.linear_forward(X, prep)
     codes = dev_u8(o["x_codes"])
     native = np.zeros(svdq.svdq_act_scales_bytes(M, K), np.uint8)
-    svdq.svdq_scales_to_native(np.ascontiguousarray(o["x_scales"]).ctypes.data, M, K, native.ctypes.data)
+    logical = np.ascontiguousarray(o["x_scales"])       # kept alive across the call
+    svdq.svdq_scales_to_native(logical.ctypes.data, M, K, native.ctypes.data)
     sc = dev_u8(native)
     D = dev_u16(o["D"]) if r else None
     Y = t.empty((M, N), dtype=t.int16, device="cuda")
@@ -266,7 +267,8 @@ def test_gemm_output_16_byte_aligned(BN, monkeypatch):
     o = ref.linear_forward(X, prep)
     codes = dev_u8(o["x_codes"])
     native = np.zeros(svdq.svdq_act_scales_bytes(M, K), np.uint8)
-    svdq.svdq_scales_to_native(np.ascontiguousarray(o["x_scales"]).ctypes.data, M, K, native.ctypes.data)
+    logical = np.ascontiguousarray(o["x_scales"])       # kept alive across the call
+    svdq.svdq_scales_to_native(logical.ctypes.data, M, K, native.ctypes.data)
     sc = dev_u8(native)
     D = dev_u16(o["D"])
     guard = 0x5A5A
