@@ -274,15 +274,33 @@ def run_native(args):
     gemm_tflops = flops / (gemm_ms * 1e-3) / 1e12
     act_bytes = M * K * 2 + K * 4 + K * r * 2 + M * K // 2 + M * K // 16 + M * r * 2
     act_gbs = act_bytes / (act_ms * 1e-3) / 1e9
-    roofline = {
-        "kernel": "fp4_gemm_kernel", "bound": "tensor", "achieved": round(gemm_tflops, 1),
-        "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(gemm_tflops / fp4_peak, 4),
+    # the GEMM's own algorithmic bytes: activation codes, scales and D in; the
+    # weight's codes, scales, L2^T and bias in; Y out
+    gemm_bytes = (M * K // 2 + M * K // 16 + M * r * 2 + N * K // 2 + N * K // 16 + N * r * 2 + N * 2
+                  + M * N * 2)
+    ridge = fp4_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)        # flop per byte
+    if flops / gemm_bytes >= ridge:
+        roofline = {
+            "kernel": "fp4_gemm_kernel", "bound": "tensor", "achieved": round(gemm_tflops, 1),
+            "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(gemm_tflops / fp4_peak, 4),
+            "peak_source": f"{peak_kind} bf16 burst {peaks['bf16_tflops']} x nominal fp4:bf16 ratio 4",
+            "frac_of_fp4_spec_9pf": round(gemm_tflops / FP4_SPEC_TFLOPS, 4),
+            "algorithmic_flops_per_launch": flops,
+        }
+    else:   # below the ridge (small M): weight streaming, against HBM
+        gemm_gbs = gemm_bytes / (gemm_ms * 1e-3) / 1e9
+        roofline = {
+            "kernel": "fp4_gemm_kernel", "bound": "hbm", "achieved": round(gemm_gbs, 1),
+            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(gemm_gbs / peaks["hbm_gbs"], 4),
+            "peak_source": f"{peak_kind} HBM copy",
+            "tflops": round(gemm_tflops, 2),
+        }
+    roofline.update({
         "traffic": _profile_traffic(GEMM_SRC, f"fp4_gemm_{args.workload}.txt"),
-        "peak_source": f"{peak_kind} bf16 burst {peaks['bf16_tflops']} x nominal fp4:bf16 ratio 4",
-        "frac_of_fp4_spec_9pf": round(gemm_tflops / FP4_SPEC_TFLOPS, 4),
-        "algorithmic_flops_per_launch": flops,
+        "algorithmic_bytes_per_launch": gemm_bytes,
+        "arithmetic_intensity_flop_per_byte": round(flops / gemm_bytes, 1),
         "launch_us": round(gemm_ms * 1e3, 2),
-    }
+    })
     act = {"kernel": "act_quant_kernel", "bound": "hbm", "achieved": round(act_gbs, 1),
            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(act_gbs / peaks["hbm_gbs"], 4),
            "algorithmic_bytes_per_launch": act_bytes, "launch_us": round(act_ms * 1e3, 2),
@@ -340,6 +358,77 @@ def run_native(args):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+    return out
+
+
+def run_block(args):
+    """The four linears of one DiT block (workloads block_<b>_{qkv,out,up,down})
+    back to back on one stream, each on its own synthetic input; one step is
+    the four layers, timed with CUDA events, L2 flushed between steps.  One GPU."""
+    import torch
+    import w4a4_rank_corrected_act_b200 as svdq
+    from workloads import gen
+
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    names = [f"block_{args.block}_{n}" for n in ("qkv", "out", "up", "down")]
+    st = torch.cuda.current_stream()
+    sh = int(st.cuda_stream)
+    layers = []
+    for nm in names:
+        spec = gen.workload(nm)
+        d = gen.make_linear(spec)
+        dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
+        lin = svdq.SvdqLinear(dev(d["W"]), torch.from_numpy(d["lam"]).cuda(), dev(d["bias"]), r=spec.r)
+        X = dev(d["X"])
+        Y = torch.empty((spec.M, spec.N), dtype=torch.int16, device="cuda")
+        nb = lin.workspace_bytes(spec.M)
+        ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+        layers.append((spec, lin, X, Y, ws, nb))
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def step(evs=None):
+        for i, (spec, lin, X, Y, ws, nb) in enumerate(layers):
+            if evs is not None:
+                evs[i].record(st)
+            svdq.svdq_linear_forward(X.data_ptr(), spec.M, lin.w, Y.data_ptr(), ws.data_ptr(), nb, sh)
+        if evs is not None:
+            evs[len(layers)].record(st)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    per = [[torch.cuda.Event(enable_timing=True) for _ in range(len(layers) + 1)] for _ in range(args.steps)]
+    with ClockSampler(0) as clk:
+        _run_for(0.5, flush, step)
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            flush.zero_()
+            step(per[i])
+        torch.cuda.synchronize()
+        _run_for(0.5, flush, step)
+    step_ms = [e[0].elapsed_time(e[-1]) for e in per]
+    layer_us = [statistics.mean(e[j].elapsed_time(e[j + 1]) for e in per) * 1e3 for j in range(len(layers))]
+    if svdq.svdq_get_device_status(sh):
+        raise SystemExit("a kernel gave up a wait")
+    flops = sum(2.0 * spec.M * spec.N * spec.K for spec, *_ in layers)
+    total_ms = sum(step_ms)
+    out = {
+        "metric": METRIC + " (DiT block: four linears)", "value": round(flops * args.steps / (total_ms * 1e-3) / 1e12, 2),
+        "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic (seeded DiT-shaped inputs; no checkpoint)",
+        "config": {"workload": f"DiT block, {layers[0][0].M} tokens: QKV 3072->9216, out 3072->3072, "
+                               "up 3072->12288, down 12288->3072, r=32, bias",
+                   "l2": "flushed between steps (256 MiB write outside the step events)",
+                   "parallelism": "replicas x1 (token-parallel, no collective)"},
+        "layers_us": {spec.name: round(t, 2) for (spec, *_), t in zip(layers, layer_us)},
+        "step_us_percentiles": {"p50": round(float(np.percentile(step_ms, 50)) * 1e3, 2),
+                                "p95": round(float(np.percentile(step_ms, 95)) * 1e3, 2)},
+        "gpu_launches": 2 * len(layers) * args.steps,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(out), flush=True)
     return out
 
 
@@ -451,6 +540,9 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-rows", type=int, default=128)
+    ap.add_argument("--block", choices=["b1", "b4"], default=None,
+                    help="time the four linears of a DiT block (QKV, out, up, down) back to back "
+                         "on one stream (b1: 4608 tokens, b4: 18432) instead of one workload")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -460,6 +552,8 @@ def main(argv=None):
         args.cpu_baseline = False
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
         raise SystemExit("for --gpus > 1 launch with torch.distributed.run (one rank per GPU)")
+    if args.block:
+        return run_block(args)
     return run_native(args)
 
 
