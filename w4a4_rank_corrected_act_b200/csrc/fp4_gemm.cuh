@@ -51,6 +51,8 @@ struct GemmParams {
   const uint8_t* x_scales;
   const uint8_t* w_scales;
   const uint16_t* bias;
+  uint16_t* Y;            // M x N bf16, row-major (the last tile's stores go straight from registers)
+  int y_align32;          // Y is 32-byte aligned: one 32-byte store per row piece
   int M, N, K, r;
   int m_tiles, n_tiles, num_tiles, kblocks;
 };
@@ -143,6 +145,76 @@ __device__ __forceinline__ void store_piece(const uint32_t (&v)[16], int slot, i
   if (lane == 0) {
     tma_store_2d(tm_y, stg_u + slot * GEMM_OUT_PIECE, n0 + c * 16, row0);
     bulk_commit_group();
+  }
+}
+
+// Bias added, rounded to bf16 and stored straight from registers: 16 columns
+// (32 bytes, one full sector) of one output row per lane, a lane per row.  The
+// bias shuffles need every lane, so the row check comes after them.
+__device__ __forceinline__ void store_piece_direct(const uint32_t (&v)[16], int c, bool has_bias,
+                                                   uint4 bias, uint16_t* yrow, bool row_ok,
+                                                   bool align32) {
+  float f[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) f[j] = __uint_as_float(v[j]);
+  if (has_bias) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int src = 2 * c + u;
+      const uint32_t bw[4] = {__shfl_sync(0xffffffffu, bias.x, src), __shfl_sync(0xffffffffu, bias.y, src),
+                              __shfl_sync(0xffffffffu, bias.z, src), __shfl_sync(0xffffffffu, bias.w, src)};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        f[u * 8 + 2 * h] += bf16_bits_to_f32(bw[h] & 0xFFFFu);
+        f[u * 8 + 2 * h + 1] += bf16_bits_to_f32(bw[h] >> 16);
+      }
+    }
+  }
+  uint32_t o[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) o[j] = pack_bf16x2(f[2 * j], f[2 * j + 1]);
+  if (!row_ok) return;
+  uint16_t* dst = yrow + c * 16;
+  if (align32) {
+    st_global_v8(dst, o);
+  } else {
+    *reinterpret_cast<uint4*>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
+    *reinterpret_cast<uint4*>(dst + 8) = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+}
+
+// Epilogue of one 128 x BN tile for the warp owning tensor-memory lanes
+// 32 q .. 32 q + 31 (= tile rows) with stores straight from registers.  Same
+// piece order and release rule as epilogue_tile (below); `yrow` is this
+// lane's output row at the tile's first column.
+template <int BN, int KOV, typename Order, typename Release>
+__device__ __forceinline__ void epilogue_tile_direct(uint32_t acc, uint32_t lane_addr, bool has_bias,
+                                                     uint4 bias, uint16_t* yrow, bool row_ok,
+                                                     bool align32, Order order, Release release) {
+  constexpr int kPieces = BN / 16;
+  static_assert(KOV % 2 == 0 && KOV < kPieces, "shared pieces: an even count below the tile's");
+  uint32_t v[2][16];
+  if constexpr (KOV > 0) {
+    uint32_t ov[KOV][16];
+#pragma unroll
+    for (int j = 0; j < KOV; ++j) tmem_ld_32x32b_x16(acc + lane_addr + order(j) * 16, ov[j]);
+    tmem_ld_wait();
+    tc_fence_before();
+    release();
+    tmem_ld_32x32b_x16(acc + lane_addr + order(KOV) * 16, v[0]);
+#pragma unroll
+    for (int j = 0; j < KOV; ++j) store_piece_direct(ov[j], order(j), has_bias, bias, yrow, row_ok, align32);
+  } else {
+    tc_fence_before();
+    release();
+    tmem_ld_32x32b_x16(acc + lane_addr + order(0) * 16, v[0]);
+  }
+  tmem_ld_wait();
+#pragma unroll 2
+  for (int i = KOV; i < kPieces; ++i) {
+    if (i + 1 < kPieces) tmem_ld_32x32b_x16(acc + lane_addr + order(i + 1) * 16, v[(i + 1) & 1]);
+    store_piece_direct(v[i & 1], order(i), has_bias, bias, yrow, row_ok, align32);
+    tmem_ld_wait();
   }
 }
 
@@ -419,13 +491,23 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       // buffer 0 shares its top columns with buffer 1, buffer 1 its bottom
       // columns with buffer 0: those pieces come first
       constexpr int kPieces = BN / 16, kOv = 2 * Cfg::kOverlapChunks;
-      epilogue_tile<BN, kOv>(
-          acc, lane_addr, lane, p.bias != nullptr, tile_bias, n0, m0 + q * 32, &tm_y, stg, stg_u,
-          [&](int i) { return buf ? i : (i + kPieces - kOv) % kPieces; },
-          [&]() {
-            __syncwarp();
-            if (lane == 0) mbar_arrive(tmem_free);
-          });
+      auto order = [&](int i) { return buf ? i : (i + kPieces - kOv) % kPieces; };
+      auto release = [&]() {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tmem_free);
+      };
+      if (t + static_cast<int>(gridDim.x) < p.num_tiles) {
+        epilogue_tile<BN, kOv>(acc, lane_addr, lane, p.bias != nullptr, tile_bias, n0, m0 + q * 32, &tm_y,
+                               stg, stg_u, order, release);
+      } else {
+        // the CTA's last tile: no MMA runs any more, so the stores go straight
+        // from registers (shorter per piece than staging + TMA; while the
+        // mainloop runs they would compete with it for the load/store unit)
+        const int row = m0 + q * 32 + lane;
+        epilogue_tile_direct<BN, kOv>(acc, lane_addr, p.bias != nullptr, tile_bias,
+                                      p.Y + static_cast<size_t>(row) * p.N + n0, row < p.M, p.y_align32 != 0,
+                                      order, release);
+      }
     }
     if (lane == 0) bulk_wait_group_all();
     __syncwarp();

@@ -368,6 +368,8 @@ svdq_status gemm_impl(const uint8_t* x_codes, const uint8_t* x_scales, const uin
   p.x_scales = x_scales;
   p.w_scales = w->w_scales;
   p.bias = w->has_bias ? w->bias : nullptr;
+  p.Y = Y;
+  p.y_align32 = (reinterpret_cast<uintptr_t>(Y) % 32) == 0;
   p.M = M;
   p.N = N;
   p.K = K;
