@@ -87,15 +87,6 @@ __global__ void __launch_bounds__(ACT_THREADS, 2)
   const int row0 = (blockIdx.x / p.ks) * ACT_ROWS;
   const int nsub = p.K / ACT_SUB / p.ks;             // sub-tiles of this CTA's K range
   const int sub0 = static_cast<int>(kpart) * nsub;   // its first sub-tile
-  if (row0 >= p.M) {
-    // rows entirely in [M, M_pad): their scale entries are written as zero
-    // (the whole cluster shares the row block, so every CTA of it leaves here)
-    for (int idx = threadIdx.x; idx < nsub * ACT_ROWS; idx += ACT_THREADS) {
-      const int g = sub0 + idx / ACT_ROWS, i = idx % ACT_ROWS;
-      *reinterpret_cast<uint32_t*>(p.x_scales + sf_offset(row0 + i, g * 4, p.K)) = 0u;
-    }
-    return;
-  }
   if (threadIdx.x == 0) *abort_flag = 0;
   const uint32_t ring = smem_u32(smem) + warp * ACT_RING * ACT_SUB_BYTES;
   auto bar = [&](int slot) { return smem_u32(bars + warp * ACT_RING + slot); };
@@ -105,9 +96,22 @@ __global__ void __launch_bounds__(ACT_THREADS, 2)
   }
   for (int c = threadIdx.x; c < 128; c += ACT_THREADS) tab[c] = e4m3_table_entry(c);
   __syncthreads();   // barriers, the E4M3 table and the abort flag are initialised
-  // the GEMM that consumes this kernel's output may be launched now: it loads
-  // weights until its griddepcontrol.wait, which waits for this grid to finish
+  // This grid may be launched while the previous kernel of the stream is still
+  // running (programmatic dependent launch): nothing in global memory is read
+  // or written before that kernel has completed.  The GEMM that consumes this
+  // kernel's output may be launched from now on: it loads weights until its
+  // own wait, which waits for this grid to finish.
+  pdl_wait();
   pdl_launch_dependents();
+  if (row0 >= p.M) {
+    // rows entirely in [M, M_pad): their scale entries are written as zero
+    // (the whole cluster shares the row block, so every CTA of it leaves here)
+    for (int idx = threadIdx.x; idx < nsub * ACT_ROWS; idx += ACT_THREADS) {
+      const int g = sub0 + idx / ACT_ROWS, i = idx % ACT_ROWS;
+      *reinterpret_cast<uint32_t*>(p.x_scales + sf_offset(row0 + i, g * 4, p.K)) = 0u;
+    }
+    return;
+  }
 
   const int my_count = nsub > warp ? (nsub - warp + ACT_WARPS - 1) / ACT_WARPS : 0;
   auto issue = [&](int jj) {

@@ -317,6 +317,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // the next kernel of the stream may be launched now; it waits for this grid
+  // before it touches global memory (see the activation kernel)
+  pdl_launch_dependents();
 
   const int kb_per_tile = p.kblocks;
   const uint32_t k_tiles64 = static_cast<uint32_t>(p.K) >> 6;

@@ -154,24 +154,24 @@ svdq_status launch_act(const CUtensorMap& tx, const ActParams& p, cudaStream_t s
   });
   if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(act)");
   const int grid = p.M_pad / ACT_ROWS * p.ks;
-  if (p.ks == 1) {
-    act_quant_kernel<R_PAD><<<grid, ACT_THREADS, smem, st>>>(tx, p);
-  } else {
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(static_cast<unsigned>(grid));
-    cfg.blockDim = dim3(ACT_THREADS);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = static_cast<unsigned>(p.ks);
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, act_quant_kernel<R_PAD>, tx, p);
-    if (e != cudaSuccess) return cuda_fail(e, "act_quant_kernel (cluster) launch");
-  }
+  // programmatic dependent launch (the kernel waits for its predecessor before
+  // touching global memory), and a cluster of ks CTAs per row block when ks > 1
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(ACT_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = static_cast<unsigned>(p.ks);
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = p.ks > 1 ? 2 : 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, act_quant_kernel<R_PAD>, tx, p);
+  if (e != cudaSuccess) return cuda_fail(e, "act_quant_kernel launch");
   SVDQ_CHECK_LAUNCH("act_quant_kernel");
   return SVDQ_OK;
 }
