@@ -178,6 +178,24 @@ svdq_status svdq_gemm(const uint8_t* x_codes, const uint8_t* x_scales, const uin
                       const svdq_weight* w, uint16_t* Y, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * The same GEMM (and whole layer, below) writing Y head-major for attention
+ * consumers: Y[h][m][d] = Yrow[m][h * head_dim + d], i.e. N / head_dim blocks
+ * of M x head_dim bf16, one per head (for a QKV projection: the Q heads, then
+ * K, then V).  The engine the chaosnode.de page ("Nunchaku Lite vs. Original")
+ * describes fuses the QKV projection with its consumers; this is the layout
+ * half of that.  head_dim % 16 == 0 and N % head_dim == 0 (INVALID_ARG
+ * otherwise).  The values are bit for bit those of svdq_gemm; the single-CTA
+ * kernel is always used.
+ * ------------------------------------------------------------------------- */
+svdq_status svdq_gemm_heads(const uint8_t* x_codes, const uint8_t* x_scales, const uint16_t* D, int M,
+                            const svdq_weight* w, int head_dim, uint16_t* Y, void* stream);
+
+/* Whole layer with head-major Y (see svdq_gemm_heads); workspace as for
+ * svdq_linear_forward. */
+svdq_status svdq_linear_forward_heads(const uint16_t* X, int M, const svdq_weight* w, int head_dim,
+                                      uint16_t* Y, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Whole layer: svdq_quantize_act then svdq_gemm on `stream`, with the
  * activation codes, scales and D placed in the caller's workspace `ws`
  * (svdq_forward_workspace_bytes(M, N, K, r) bytes, device).

@@ -57,6 +57,8 @@ SIGNATURES = {
     "svdq_linear_forward": (_I, [_P, _I, _WP, _P, _P, _SZ, _P]),
     "svdq_linear_forward_host": (_I, [_P, _I, _WP, _P, _P, _P, _P, _SZ, _P]),
     "svdq_linear_forward_noalloc": (_I, [_P, _I, _WP, _P, _P]),
+    "svdq_gemm_heads": (_I, [_P, _P, _P, _I, _WP, _I, _P, _P]),
+    "svdq_linear_forward_heads": (_I, [_P, _I, _WP, _I, _P, _P, _SZ, _P]),
     "svdq_weight_export": (_I, [_WP, _P, _P, _P, _P, _P, _P]),
     "svdq_weight_import": (_I, [_WP, _P, _P, _P, _P, _P, _P, _P]),
     "svdq_calib_absmax": (_I, [_P, _I, _I, _P, _P]),
@@ -164,6 +166,16 @@ def svdq_gemm(x_codes: int, x_scales: int, D: int, M: int, w: svdq_weight, Y: in
 def svdq_linear_forward(X: int, M: int, w: svdq_weight, Y: int, ws: int, ws_bytes: int,
                         stream: int) -> None:
     _call("svdq_linear_forward", X, M, ctypes.byref(w), Y, ws, ws_bytes, stream or None)
+
+
+def svdq_gemm_heads(x_codes: int, x_scales: int, D: int, M: int, w: svdq_weight, head_dim: int,
+                    Y: int, stream: int) -> None:
+    _call("svdq_gemm_heads", x_codes, x_scales, D or None, M, ctypes.byref(w), head_dim, Y, stream or None)
+
+
+def svdq_linear_forward_heads(X: int, M: int, w: svdq_weight, head_dim: int, Y: int, ws: int,
+                              ws_bytes: int, stream: int) -> None:
+    _call("svdq_linear_forward_heads", X, M, ctypes.byref(w), head_dim, Y, ws, ws_bytes, stream or None)
 
 
 def svdq_linear_forward_host(X_host: int, M: int, w: svdq_weight, Y_host: int, X_dev: int,

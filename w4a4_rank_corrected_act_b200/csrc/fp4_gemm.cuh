@@ -53,6 +53,7 @@ struct GemmParams {
   const uint16_t* bias;
   uint16_t* Y;            // M x N bf16, row-major (the last tile's stores go straight from registers)
   int y_align32;          // Y is 32-byte aligned: one 32-byte store per row piece
+  int head_dim;           // 0: Y row-major; else Y head-major, [N / head_dim][M][head_dim]
   int M, N, K, r;
   int m_tiles, n_tiles, num_tiles, kblocks;
 };
@@ -110,7 +111,8 @@ __device__ __forceinline__ uint4 load_tile_bias(const uint16_t* bias, int n0, in
 // TMA.  A store may still be reading the other buffer.
 __device__ __forceinline__ void store_piece(const uint32_t (&v)[16], int slot, int c, int lane,
                                             bool has_bias, uint4 bias, int n0, int row0,
-                                            const CUtensorMap* tm_y, uint8_t* stg, uint32_t stg_u) {
+                                            const CUtensorMap* tm_y, uint8_t* stg, uint32_t stg_u,
+                                            int head_dim) {
   float f[16];
 #pragma unroll
   for (int j = 0; j < 16; ++j) f[j] = __uint_as_float(v[j]);
@@ -143,7 +145,10 @@ __device__ __forceinline__ void store_piece(const uint32_t (&v)[16], int slot, i
   fence_proxy_async_smem();
   __syncwarp();
   if (lane == 0) {
-    tma_store_2d(tm_y, stg_u + slot * GEMM_OUT_PIECE, n0 + c * 16, row0);
+    // row-major Y: (column, row); head-major Y: (column in head, row, head)
+    const int n = n0 + c * 16;
+    if (head_dim == 0) tma_store_2d(tm_y, stg_u + slot * GEMM_OUT_PIECE, n, row0);
+    else tma_store_3d(tm_y, stg_u + slot * GEMM_OUT_PIECE, n % head_dim, row0, n / head_dim);
     bulk_commit_group();
   }
 }
@@ -152,7 +157,7 @@ __device__ __forceinline__ void store_piece(const uint32_t (&v)[16], int slot, i
 // (32 bytes, one full sector) of one output row per lane, a lane per row.  The
 // bias shuffles need every lane, so the row check comes after them.
 __device__ __forceinline__ void store_piece_direct(const uint32_t (&v)[16], int c, bool has_bias,
-                                                   uint4 bias, uint16_t* yrow, bool row_ok,
+                                                   uint4 bias, uint16_t* dst, bool row_ok,
                                                    bool align32) {
   float f[16];
 #pragma unroll
@@ -174,7 +179,6 @@ __device__ __forceinline__ void store_piece_direct(const uint32_t (&v)[16], int 
 #pragma unroll
   for (int j = 0; j < 8; ++j) o[j] = pack_bf16x2(f[2 * j], f[2 * j + 1]);
   if (!row_ok) return;
-  uint16_t* dst = yrow + c * 16;
   if (align32) {
     st_global_v8(dst, o);
   } else {
@@ -187,9 +191,9 @@ __device__ __forceinline__ void store_piece_direct(const uint32_t (&v)[16], int 
 // 32 q .. 32 q + 31 (= tile rows) with stores straight from registers.  Same
 // piece order and release rule as epilogue_tile (below); `yrow` is this
 // lane's output row at the tile's first column.
-template <int BN, int KOV, typename Order, typename Release>
+template <int BN, int KOV, typename Order, typename Release, typename Dst>
 __device__ __forceinline__ void epilogue_tile_direct(uint32_t acc, uint32_t lane_addr, bool has_bias,
-                                                     uint4 bias, uint16_t* yrow, bool row_ok,
+                                                     uint4 bias, Dst dst, bool row_ok,
                                                      bool align32, Order order, Release release) {
   constexpr int kPieces = BN / 16;
   static_assert(KOV % 2 == 0 && KOV < kPieces, "shared pieces: an even count below the tile's");
@@ -203,7 +207,7 @@ __device__ __forceinline__ void epilogue_tile_direct(uint32_t acc, uint32_t lane
     release();
     tmem_ld_32x32b_x16(acc + lane_addr + order(KOV) * 16, v[0]);
 #pragma unroll
-    for (int j = 0; j < KOV; ++j) store_piece_direct(ov[j], order(j), has_bias, bias, yrow, row_ok, align32);
+    for (int j = 0; j < KOV; ++j) store_piece_direct(ov[j], order(j), has_bias, bias, dst(order(j)), row_ok, align32);
   } else {
     tc_fence_before();
     release();
@@ -213,7 +217,7 @@ __device__ __forceinline__ void epilogue_tile_direct(uint32_t acc, uint32_t lane
 #pragma unroll 2
   for (int i = KOV; i < kPieces; ++i) {
     if (i + 1 < kPieces) tmem_ld_32x32b_x16(acc + lane_addr + order(i + 1) * 16, v[(i + 1) & 1]);
-    store_piece_direct(v[i & 1], order(i), has_bias, bias, yrow, row_ok, align32);
+    store_piece_direct(v[i & 1], order(i), has_bias, bias, dst(order(i)), row_ok, align32);
     tmem_ld_wait();
   }
 }
@@ -228,7 +232,7 @@ template <int BN, int KOV, typename Order, typename Release>
 __device__ __forceinline__ void epilogue_tile(uint32_t acc, uint32_t lane_addr, int lane,
                                               bool has_bias, uint4 bias, int n0, int row0,
                                               const CUtensorMap* tm_y, uint8_t* stg, uint32_t stg_u,
-                                              Order order, Release release) {
+                                              Order order, Release release, int head_dim = 0) {
   constexpr int kPieces = BN / 16;
   static_assert(KOV % 2 == 0 && KOV < kPieces, "shared pieces: an even count below the tile's");
   uint32_t v[2][16];
@@ -242,7 +246,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t acc, uint32_t lane_addr, 
     tmem_ld_32x32b_x16(acc + lane_addr + order(KOV) * 16, v[0]);
 #pragma unroll
     for (int j = 0; j < KOV; ++j)
-      store_piece(ov[j], j & 1, order(j), lane, has_bias, bias, n0, row0, tm_y, stg, stg_u);
+      store_piece(ov[j], j & 1, order(j), lane, has_bias, bias, n0, row0, tm_y, stg, stg_u, head_dim);
   } else {
     tc_fence_before();
     release();
@@ -252,7 +256,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t acc, uint32_t lane_addr, 
 #pragma unroll 2
   for (int i = KOV; i < kPieces; ++i) {
     if (i + 1 < kPieces) tmem_ld_32x32b_x16(acc + lane_addr + order(i + 1) * 16, v[(i + 1) & 1]);
-    store_piece(v[i & 1], i & 1, order(i), lane, has_bias, bias, n0, row0, tm_y, stg, stg_u);
+    store_piece(v[i & 1], i & 1, order(i), lane, has_bias, bias, n0, row0, tm_y, stg, stg_u, head_dim);
     tmem_ld_wait();
   }
 }
@@ -501,15 +505,20 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       };
       if (t + static_cast<int>(gridDim.x) < p.num_tiles) {
         epilogue_tile<BN, kOv>(acc, lane_addr, lane, p.bias != nullptr, tile_bias, n0, m0 + q * 32, &tm_y,
-                               stg, stg_u, order, release);
+                               stg, stg_u, order, release, p.head_dim);
       } else {
         // the CTA's last tile: no MMA runs any more, so the stores go straight
         // from registers (shorter per piece than staging + TMA; while the
         // mainloop runs they would compete with it for the load/store unit)
         const int row = m0 + q * 32 + lane;
-        epilogue_tile_direct<BN, kOv>(acc, lane_addr, p.bias != nullptr, tile_bias,
-                                      p.Y + static_cast<size_t>(row) * p.N + n0, row < p.M, p.y_align32 != 0,
-                                      order, release);
+        auto dst = [&](int c) {
+          const int n = n0 + c * 16;
+          return p.head_dim == 0
+                     ? p.Y + static_cast<size_t>(row) * p.N + n
+                     : p.Y + (static_cast<size_t>(n / p.head_dim) * p.M + row) * p.head_dim + n % p.head_dim;
+        };
+        epilogue_tile_direct<BN, kOv>(acc, lane_addr, p.bias != nullptr, tile_bias, dst, row < p.M,
+                                      p.y_align32 != 0, order, release);
       }
     }
     if (lane == 0) bulk_wait_group_all();

@@ -129,6 +129,33 @@ svdq_status make_tmap(CUtensorMap* m, CUtensorMapDataType dt, const void* base, 
   return SVDQ_OK;
 }
 
+// Head-major output [heads][M][head_dim] bf16, stored in 16-column x 32-row
+// pieces through the same 32-byte-swizzled staging as the row-major map.
+svdq_status make_tmap_heads(CUtensorMap* m, const void* base, int head_dim, int M, int heads) {
+  auto fn = encode_fn();
+  if (fn == nullptr) {
+    g_last_error = "cuTensorMapEncodeTiled entry point unavailable";
+    return SVDQ_ERR_CUDA;
+  }
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(M),
+                        static_cast<cuuint64_t>(heads)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * 2,
+                           static_cast<cuuint64_t>(head_dim) * 2 * static_cast<cuuint64_t>(M)};
+  cuuint32_t box[3] = {16, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    char buf[160];
+    std::snprintf(buf, sizeof(buf), "cuTensorMapEncodeTiled (heads) failed (%d) head_dim=%d M=%d heads=%d",
+                  static_cast<int>(r), head_dim, M, heads);
+    g_last_error = buf;
+    return SVDQ_ERR_CUDA;
+  }
+  return SVDQ_OK;
+}
+
 CUtensorMapSwizzle lr_swizzle(int r_pad) {
   return r_pad == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
                      : r_pad == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
@@ -329,9 +356,10 @@ svdq_status gemm_pair_impl(const uint8_t* x_codes, const uint8_t* x_scales, cons
   }
 }
 
+// head_dim == 0: Y row-major M x N; else Y head-major [N / head_dim][M][head_dim]
 svdq_status gemm_impl(const uint8_t* x_codes, const uint8_t* x_scales, const uint16_t* D, int M,
-                      const svdq_weight* w, uint16_t* Y, cudaStream_t st) {
-  {
+                      const svdq_weight* w, uint16_t* Y, cudaStream_t st, int head_dim = 0) {
+  if (head_dim == 0) {
     // the CTA-pair kernel (256 x 256 tiles) is used on request (SVDQ_GEMM_PAIR=1)
     bool pair = false;
     if (const char* e = std::getenv("SVDQ_GEMM_PAIR")) pair = (std::atoi(e) != 0) && (w->N % 256 == 0);
@@ -353,8 +381,11 @@ svdq_status gemm_impl(const uint8_t* x_codes, const uint8_t* x_scales, const uin
   s = make_tmap(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->w_codes, K / 2, N, K / 2, 128, BN,
                 CU_TENSOR_MAP_SWIZZLE_128B);
   if (s != SVDQ_OK) return s;
-  s = make_tmap(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, N, M, static_cast<uint64_t>(N) * 2, 16, 32,
-                CU_TENSOR_MAP_SWIZZLE_32B);
+  if (head_dim == 0)
+    s = make_tmap(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, N, M, static_cast<uint64_t>(N) * 2, 16, 32,
+                  CU_TENSOR_MAP_SWIZZLE_32B);
+  else
+    s = make_tmap_heads(&ty, Y, head_dim, M, N / head_dim);
   if (s != SVDQ_OK) return s;
   if (r > 0) {
     s = make_tmap(&td, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, D, r, M, static_cast<uint64_t>(r) * 2, rp,
@@ -370,6 +401,7 @@ svdq_status gemm_impl(const uint8_t* x_codes, const uint8_t* x_scales, const uin
   p.bias = w->has_bias ? w->bias : nullptr;
   p.Y = Y;
   p.y_align32 = (reinterpret_cast<uintptr_t>(Y) % 32) == 0;
+  p.head_dim = head_dim;
   p.M = M;
   p.N = N;
   p.K = K;
@@ -838,6 +870,36 @@ svdq_status svdq_linear_forward(const uint16_t* X, int M, const svdq_weight* w, 
   s = quantize_act_impl(X, M, w, a.codes, a.scales, a.D, st);
   if (s != SVDQ_OK) return s;
   return gemm_impl(a.codes, a.scales, a.D, M, w, Y, st);
+}
+
+svdq_status svdq_gemm_heads(const uint8_t* x_codes, const uint8_t* x_scales, const uint16_t* D, int M,
+                            const svdq_weight* w, int head_dim, uint16_t* Y, void* stream) {
+  svdq_status s = check_weight(w);
+  if (s != SVDQ_OK) return s;
+  if (M < 0 || head_dim <= 0 || head_dim % 16 != 0 || w->N % head_dim != 0) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  if (x_codes == nullptr || x_scales == nullptr || Y == nullptr || (w->r > 0 && D == nullptr))
+    return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(x_codes) || !aligned16(x_scales) || !aligned16(Y) || (w->r > 0 && !aligned16(D)))
+    return SVDQ_ERR_MISALIGNED;
+  return gemm_impl(x_codes, x_scales, D, M, w, Y, static_cast<cudaStream_t>(stream), head_dim);
+}
+
+svdq_status svdq_linear_forward_heads(const uint16_t* X, int M, const svdq_weight* w, int head_dim,
+                                      uint16_t* Y, void* ws, size_t ws_bytes, void* stream) {
+  svdq_status s = check_weight(w);
+  if (s != SVDQ_OK) return s;
+  if (M < 0 || head_dim <= 0 || head_dim % 16 != 0 || w->N % head_dim != 0) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  if (X == nullptr || Y == nullptr || ws == nullptr) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(Y) || !aligned16(ws)) return SVDQ_ERR_MISALIGNED;
+  if (ws_bytes < act_ws_layout(M, w->K, w->r, nullptr, nullptr)) return SVDQ_ERR_WORKSPACE_TOO_SMALL;
+  ActWs a;
+  act_ws_layout(M, w->K, w->r, static_cast<uint8_t*>(ws), &a);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  s = quantize_act_impl(X, M, w, a.codes, a.scales, a.D, st);
+  if (s != SVDQ_OK) return s;
+  return gemm_impl(a.codes, a.scales, a.D, M, w, Y, st, head_dim);
 }
 
 svdq_status svdq_linear_forward_host(const uint16_t* X_host, int M, const svdq_weight* w,
