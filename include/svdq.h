@@ -205,8 +205,13 @@ svdq_status svdq_linear_forward(const uint16_t* X, int M, const svdq_weight* w, 
 
 /* Same as svdq_linear_forward but with X and Y in pinned HOST memory: copies
  * X_host -> X_dev (M x K bf16), runs the layer into Y_dev, copies Y_dev ->
- * Y_host (M x N bf16), all asynchronously on `stream` (the caller
- * synchronises before reading Y_host). */
+ * Y_host (M x N bf16), asynchronously with respect to the host and ordered on
+ * `stream` (the caller synchronises `stream` before reading Y_host).  Above
+ * 1024 rows the work is split into chunks of 1024 rows: each chunk's copy
+ * back to the host runs on a second, library-owned stream (one per device,
+ * created on first use) while the next chunk is copied in and computed, and
+ * `stream` then waits for the last copy.  ws is sized for M as for
+ * svdq_linear_forward. */
 svdq_status svdq_linear_forward_host(const uint16_t* X_host, int M, const svdq_weight* w,
                                      uint16_t* Y_host, uint16_t* X_dev, uint16_t* Y_dev,
                                      void* ws, size_t ws_bytes, void* stream);

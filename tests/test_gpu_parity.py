@@ -322,9 +322,13 @@ def test_forward_small_workload_end_to_end():
     assert np.max(np.abs(ref.bf16_to_f64(Y) - own)) <= 2e-2 * rms * 10  # loose cross-check
 
 
-def test_forward_host_buffers_match_device_path():
+@pytest.mark.parametrize("M", [200, 2600])
+def test_forward_host_buffers_match_device_path(M):
+    """Host-buffer forward; M = 2600 takes the pipelined path (chunks of 1024
+    rows, copies back on a second stream), and only the caller's stream is
+    synchronised before Y is read."""
     t = torch()
-    M, K, N, r = 200, 512, 384, 32
+    K, N, r = 512, 384, 32
     X, W, B, lam = _inputs(M, K, N, seed=91)
     lin, _ = _prepare(W, lam, B, r)
     Yd = to_np_u16(lin.forward(dev_u16(X).view(t.bfloat16)).view(t.int16))
@@ -334,9 +338,10 @@ def test_forward_host_buffers_match_device_path():
     Ydev = t.empty((M, N), dtype=t.int16, device="cuda")
     nb = lin.workspace_bytes(M)
     ws = empty_u8(nb)
+    t.cuda.synchronize()
     svdq.svdq_linear_forward_host(Xh.data_ptr(), M, lin.w, Yh.data_ptr(), Xdev.data_ptr(),
                                   Ydev.data_ptr(), ws.data_ptr(), nb, stream())
-    t.cuda.synchronize()
+    t.cuda.current_stream().synchronize()
     assert np.array_equal(Yh.numpy().view(np.uint16), Yd)
 
 

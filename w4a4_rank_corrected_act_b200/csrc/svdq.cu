@@ -902,6 +902,33 @@ svdq_status svdq_linear_forward_heads(const uint16_t* X, int M, const svdq_weigh
   return gemm_impl(a.codes, a.scales, a.D, M, w, Y, st, head_dim);
 }
 
+// Copy-out stream and events of the host-buffer path, created once per device.
+struct HostPipe {
+  static constexpr int kEvents = 8;
+  cudaStream_t out = nullptr;
+  cudaEvent_t ev[kEvents] = {};
+  cudaEvent_t done = nullptr;
+  bool ready = false;
+};
+
+svdq_status host_pipe(HostPipe** out) {
+  static std::mutex mu;
+  static HostPipe pipes[16];
+  int dev = 0;
+  SVDQ_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 16) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  std::lock_guard<std::mutex> lock(mu);
+  HostPipe& hp = pipes[dev];
+  if (!hp.ready) {
+    SVDQ_CUDA(cudaStreamCreateWithFlags(&hp.out, cudaStreamNonBlocking));
+    for (auto& e : hp.ev) SVDQ_CUDA(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+    SVDQ_CUDA(cudaEventCreateWithFlags(&hp.done, cudaEventDisableTiming));
+    hp.ready = true;
+  }
+  *out = &hp;
+  return SVDQ_OK;
+}
+
 svdq_status svdq_linear_forward_host(const uint16_t* X_host, int M, const svdq_weight* w,
                                      uint16_t* Y_host, uint16_t* X_dev, uint16_t* Y_dev, void* ws,
                                      size_t ws_bytes, void* stream) {
@@ -909,12 +936,42 @@ svdq_status svdq_linear_forward_host(const uint16_t* X_host, int M, const svdq_w
   if (s != SVDQ_OK) return s;
   if (M < 0) return SVDQ_ERR_INVALID_ARG;
   if (M == 0) return SVDQ_OK;
-  if (X_host == nullptr || Y_host == nullptr) return SVDQ_ERR_INVALID_ARG;
+  if (X_host == nullptr || Y_host == nullptr || X_dev == nullptr || Y_dev == nullptr || ws == nullptr)
+    return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(X_dev) || !aligned16(Y_dev) || !aligned16(ws)) return SVDQ_ERR_MISALIGNED;
+  if (ws_bytes < act_ws_layout(M, w->K, w->r, nullptr, nullptr)) return SVDQ_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  SVDQ_CUDA(cudaMemcpyAsync(X_dev, X_host, static_cast<size_t>(M) * w->K * 2, cudaMemcpyHostToDevice, st));
-  s = svdq_linear_forward(X_dev, M, w, Y_dev, ws, ws_bytes, stream);
+  const size_t K = w->K, N = w->N;
+  constexpr int kChunk = 1024;   // token rows per pipelined chunk (a multiple of 128)
+  if (M <= kChunk) {
+    SVDQ_CUDA(cudaMemcpyAsync(X_dev, X_host, static_cast<size_t>(M) * K * 2, cudaMemcpyHostToDevice, st));
+    s = svdq_linear_forward(X_dev, M, w, Y_dev, ws, ws_bytes, stream);
+    if (s != SVDQ_OK) return s;
+    SVDQ_CUDA(cudaMemcpyAsync(Y_host, Y_dev, static_cast<size_t>(M) * N * 2, cudaMemcpyDeviceToHost, st));
+    return SVDQ_OK;
+  }
+  // Chunks of rows (rows are independent): X in and the layer run on `stream`,
+  // Y out on a second stream, so that chunk i's copy to the host overlaps the
+  // copy in and the layer of chunk i + 1.  `stream` finally waits for the last
+  // copy out, so the call stays asynchronous and ordered on `stream`.
+  HostPipe* hp = nullptr;
+  s = host_pipe(&hp);
   if (s != SVDQ_OK) return s;
-  SVDQ_CUDA(cudaMemcpyAsync(Y_host, Y_dev, static_cast<size_t>(M) * w->N * 2, cudaMemcpyDeviceToHost, st));
+  int i = 0;
+  for (int r0 = 0; r0 < M; r0 += kChunk, ++i) {
+    const int rows = std::min(kChunk, M - r0);
+    SVDQ_CUDA(cudaMemcpyAsync(X_dev + r0 * K, X_host + r0 * K, static_cast<size_t>(rows) * K * 2,
+                              cudaMemcpyHostToDevice, st));
+    s = svdq_linear_forward(X_dev + r0 * K, rows, w, Y_dev + r0 * N, ws, ws_bytes, stream);
+    if (s != SVDQ_OK) return s;
+    cudaEvent_t ev = hp->ev[i % HostPipe::kEvents];
+    SVDQ_CUDA(cudaEventRecord(ev, st));
+    SVDQ_CUDA(cudaStreamWaitEvent(hp->out, ev, 0));
+    SVDQ_CUDA(cudaMemcpyAsync(Y_host + r0 * N, Y_dev + r0 * N, static_cast<size_t>(rows) * N * 2,
+                              cudaMemcpyDeviceToHost, hp->out));
+  }
+  SVDQ_CUDA(cudaEventRecord(hp->done, hp->out));
+  SVDQ_CUDA(cudaStreamWaitEvent(st, hp->done, 0));
   return SVDQ_OK;
 }
 
