@@ -8,13 +8,16 @@ bits, subnormal step 2^-9, largest finite 448; bf16: 8 significant bits) with
 Python's round(), which rounds half to even.  Float32 operations are done on
 np.float32 scalars (IEEE single, round to nearest even).
 
-It follows the same readings R1-R9 as ``oracle/svdq_ref.py`` (see there).  It
-takes L1/L2 as given: the SVD itself is pinned by the textbook identities in
-the tests, not re-derived here.
+It follows the same readings R1-R9 as ``oracle/svdq_ref.py`` (see there), and
+for the INT4 variant R15-R18 of ``oracle/int4_ref.py``, where half precision
+is rounded with Python's own binary16 packing (struct format "e", round half
+to even) instead of NumPy's.  It takes L1/L2 as given: the SVD itself is
+pinned by the textbook identities in the tests, not re-derived here.
 """
 from __future__ import annotations
 
 import math
+import struct
 
 import numpy as np
 
@@ -109,20 +112,40 @@ def _bf(bits) -> float:
     return float(np.array([int(bits) << 16], dtype=np.uint32).view(np.float32)[0])
 
 
-def forward(X_bits, W_bits, lam, bias_bits, L1_bits, L2_bits):
-    """Whole layer on tiny inputs with explicit loops.
+def f16_round(x: float) -> float:
+    """Nearest binary16 value of a non-negative float (ties to even), saturating
+    at 65504, by Python's struct packing."""
+    return struct.unpack("<e", struct.pack("<e", min(x, 65504.0)))[0]
 
-    X_bits M x K, W_bits N x K (bf16 bits), lam K (float32), bias_bits N or None,
-    L1_bits K x r, L2_bits r x N (bf16 bits).  Returns a dict with unpacked x/w
-    codes, x/w scale codes, D (bf16 values, M x r) and Y64 (float64, M x N).
-    """
+
+def quantize_row_int4(vals):
+    """One row of float32 values -> (list of int codes in [-8, 7], list of fp16 scale values)."""
+    K = len(vals)
+    codes, scales = [], []
+    for g in range(K // 64):
+        grp = [F32(vals[g * 64 + i]) for i in range(64)]
+        a = F32(0)
+        for v in grp:
+            a = max(a, F32(abs(v)))
+        s = f16_round(float(F32(a) / F32(7)))
+        scales.append(s)
+        for v in grp:
+            if s == 0.0:
+                codes.append(0)
+            else:
+                q = round(float(F32(v) / F32(s)))     # half to even
+                codes.append(max(-8, min(7, q)))
+    return codes, scales
+
+
+def _forward(X_bits, W_bits, lam, bias_bits, L1_bits, L2_bits, quantize, deq_x):
     M, K = len(X_bits), len(X_bits[0])
     N = len(W_bits)
     r = len(L1_bits[0]) if K and len(L1_bits) else 0
     inv = [F32(1) / F32(lam[k]) for k in range(K)]
     # activation side
     xhat = [[F32(F32(_bf(X_bits[m][k])) * inv[k]) for k in range(K)] for m in range(M)]
-    xq = [quantize_row(row) for row in xhat]
+    xq = [quantize(row) for row in xhat]
     # low-rank down projection, f64 sum of bf16 x bf16 products
     L1 = [[_bf(L1_bits[k][j]) for j in range(r)] for k in range(K)]
     L2 = [[_bf(L2_bits[j][n]) for n in range(N)] for j in range(r)]
@@ -145,7 +168,7 @@ def forward(X_bits, W_bits, lam, bias_bits, L1_bits, L2_bits):
             for j in range(r):
                 acc += L1[k][j] * L2[j][n]
             rrow.append(F32(float(what) - acc))
-        wq.append(quantize_row(rrow))
+        wq.append(quantize(rrow))
     # output in float64
     Y = []
     for m in range(M):
@@ -153,9 +176,7 @@ def forward(X_bits, W_bits, lam, bias_bits, L1_bits, L2_bits):
         for n in range(N):
             acc = 0.0
             for k in range(K):
-                xa = code_value(xq[m][0][k]) * e4m3_value(xq[m][1][k // 16])
-                wb = code_value(wq[n][0][k]) * e4m3_value(wq[n][1][k // 16])
-                acc += xa * wb
+                acc += deq_x(xq[m], k) * deq_x(wq[n], k)
             for j in range(r):
                 acc += D[m][j] * L2[j][n]
             if bias_bits is not None:
@@ -164,3 +185,22 @@ def forward(X_bits, W_bits, lam, bias_bits, L1_bits, L2_bits):
         Y.append(yrow)
     return dict(x_codes=[q[0] for q in xq], x_scales=[q[1] for q in xq],
                 w_codes=[q[0] for q in wq], w_scales=[q[1] for q in wq], D=D, Y64=Y)
+
+
+def forward(X_bits, W_bits, lam, bias_bits, L1_bits, L2_bits):
+    """Whole NVFP4 layer on tiny inputs with explicit loops.
+
+    X_bits M x K, W_bits N x K (bf16 bits), lam K (float32), bias_bits N or None,
+    L1_bits K x r, L2_bits r x N (bf16 bits).  Returns a dict with unpacked x/w
+    codes, x/w scale codes, D (bf16 values, M x r) and Y64 (float64, M x N).
+    """
+    return _forward(X_bits, W_bits, lam, bias_bits, L1_bits, L2_bits, quantize_row,
+                    lambda q, k: code_value(q[0][k]) * e4m3_value(q[1][k // 16]))
+
+
+def forward_int4(X_bits, W_bits, lam, bias_bits, L1_bits, L2_bits):
+    """Whole INT4 layer on tiny inputs (K a multiple of 64) with explicit loops;
+    same arguments and result fields as forward(), the codes as signed ints and
+    the scales as fp16 values."""
+    return _forward(X_bits, W_bits, lam, bias_bits, L1_bits, L2_bits, quantize_row_int4,
+                    lambda q, k: q[0][k] * q[1][k // 64])
