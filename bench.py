@@ -15,6 +15,10 @@ Multi-GPU (torchrun, one rank per GPU): the layer is run as independent
 replicas (token-parallel data parallelism, weights replicated, no collective on
 the data path); value = all ranks' flops / max-over-ranks device time.
 
+``--format int4`` runs the same step with the layer's INT4 variant (signed
+4-bit codes, fp16 scale per 64 elements; integer group sums on the 8-bit
+integer warp MMA) and reports it against the 8-bit integer tensor peak.
+
 ``--impl reference`` times the CPU oracle (the only other implementation of the
 method available) on the host cores, on a bounded row sample of the same
 workload, and prints the same JSON line with "impl": "reference".
@@ -45,6 +49,8 @@ _CSRC = os.path.join(ROOT, "w4a4_rank_corrected_act_b200", "csrc")
 # the sources each kernel is compiled from (a profile is stale once any changed)
 GEMM_SRC = [os.path.join(_CSRC, f) for f in ("fp4_gemm.cuh", "ptx.cuh", "nvfp4.cuh")]
 ACT_SRC = [os.path.join(_CSRC, f) for f in ("act_quant.cuh", "ptx.cuh", "nvfp4.cuh")]
+INT4_SRC = [os.path.join(_CSRC, f) for f in ("int4.cuh", "act_quant.cuh", "ptx.cuh", "nvfp4.cuh")]
+I8_OVER_BF16 = 2.0                # nominal dense ratio int8 : bf16 (4.5 / 2.25 POPS)
 
 
 def _peaks():
@@ -203,7 +209,9 @@ def run_native(args):
     def dev(a):
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
 
-    lin = svdq.SvdqLinear(dev(d["W"]), torch.from_numpy(d["lam"]).cuda(), dev(d["bias"]), r=r)
+    int4 = args.format == "int4"
+    lin = svdq.SvdqLinear(dev(d["W"]), torch.from_numpy(d["lam"]).cuda(), dev(d["bias"]), r=r,
+                          format=args.format)
     X = dev(d["X"])
     Y = torch.empty((M, N), dtype=torch.int16, device="cuda")
     nb = lin.workspace_bytes(M)
@@ -272,14 +280,24 @@ def run_native(args):
     peaks, peak_kind = _peaks()
     fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
     gemm_tflops = flops / (gemm_ms * 1e-3) / 1e12
-    act_bytes = M * K * 2 + K * 4 + K * r * 2 + M * K // 2 + M * K // 16 + M * r * 2
+    # scale bytes per element: one E4M3 per 16 (NVFP4) or one fp16 per 64 (INT4)
+    sc_div = 32 if int4 else 16
+    act_bytes = M * K * 2 + K * 4 + K * r * 2 + M * K // 2 + M * K // sc_div + M * r * 2
     act_gbs = act_bytes / (act_ms * 1e-3) / 1e9
     # the GEMM's own algorithmic bytes: activation codes, scales and D in; the
     # weight's codes, scales, L2^T and bias in; Y out
-    gemm_bytes = (M * K // 2 + M * K // 16 + M * r * 2 + N * K // 2 + N * K // 16 + N * r * 2 + N * 2
-                  + M * N * 2)
+    gemm_bytes = (M * K // 2 + M * K // sc_div + M * r * 2 + N * K // 2 + N * K // sc_div + N * r * 2
+                  + N * 2 + M * N * 2)
     ridge = fp4_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)        # flop per byte
-    if flops / gemm_bytes >= ridge:
+    if int4:
+        i8_peak = peaks["bf16_tflops"] * I8_OVER_BF16
+        roofline = {
+            "kernel": "int4_gemm_kernel", "bound": "tensor", "achieved": round(gemm_tflops, 1),
+            "peak": round(i8_peak, 1), "unit": "TFLOP/s", "frac": round(gemm_tflops / i8_peak, 4),
+            "peak_source": f"{peak_kind} bf16 burst {peaks['bf16_tflops']} x nominal int8:bf16 ratio 2",
+            "algorithmic_flops_per_launch": flops,
+        }
+    elif flops / gemm_bytes >= ridge:
         roofline = {
             "kernel": "fp4_gemm_kernel", "bound": "tensor", "achieved": round(gemm_tflops, 1),
             "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(gemm_tflops / fp4_peak, 4),
@@ -296,15 +314,18 @@ def run_native(args):
             "tflops": round(gemm_tflops, 2),
         }
     roofline.update({
-        "traffic": _profile_traffic(GEMM_SRC, f"fp4_gemm_{args.workload}.txt"),
+        "traffic": (_profile_traffic(INT4_SRC, f"int4_gemm_{args.workload}.txt") if int4 else
+                    _profile_traffic(GEMM_SRC, f"fp4_gemm_{args.workload}.txt")),
         "algorithmic_bytes_per_launch": gemm_bytes,
         "arithmetic_intensity_flop_per_byte": round(flops / gemm_bytes, 1),
         "launch_us": round(gemm_ms * 1e3, 2),
     })
-    act = {"kernel": "act_quant_kernel", "bound": "hbm", "achieved": round(act_gbs, 1),
+    act = {"kernel": "act_quant_int4_kernel" if int4 else "act_quant_kernel", "bound": "hbm",
+           "achieved": round(act_gbs, 1),
            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(act_gbs / peaks["hbm_gbs"], 4),
            "algorithmic_bytes_per_launch": act_bytes, "launch_us": round(act_ms * 1e3, 2),
-           "traffic": _profile_traffic(ACT_SRC, f"act_quant_{args.workload}.txt")}
+           "traffic": (_profile_traffic(INT4_SRC, f"act_quant_int4_{args.workload}.txt") if int4 else
+                       _profile_traffic(ACT_SRC, f"act_quant_{args.workload}.txt"))}
 
     # end to end through the public API with host buffers (pinned), per step:
     # H2D of X, the layer, D2H of Y
@@ -335,14 +356,15 @@ def run_native(args):
             "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "nvfp4", "data": "synthetic (seeded DiT-shaped inputs; no checkpoint)",
+            "dtype": "int4" if int4 else "nvfp4",
+            "data": "synthetic (seeded DiT-shaped inputs; no checkpoint)",
             "config": {"workload": f"{spec.name}: DiT joint-attention QKV projection at 1024x1024"
                                    if spec.name == "qkv" else spec.name,
-                       "M": M, "K": K, "N": N, "r": r, "bias": True,
+                       "M": M, "K": K, "N": N, "r": r, "bias": True, "format": args.format,
                        "l2": "flushed between steps (256 MiB write outside the step events)",
                        "parallelism": f"replicas x{world} (token-parallel, no collective)"},
             "pct_fp4_peak": {"of_spec_9000": round(value / FP4_SPEC_TFLOPS, 4),
-                             "of_measured_bf16x4": round(value / fp4_peak, 4)},
+                             "of_measured_bf16x4": round(value / fp4_peak, 4)} if not int4 else None,
             "us_per_layer": round(ms_per_step * 1e3, 2),
             "step_us_percentiles": {"p50": round(float(np.percentile(step_ms, 50)) * 1e3, 2),
                                     "p95": round(float(np.percentile(step_ms, 95)) * 1e3, 2)},
@@ -353,7 +375,8 @@ def run_native(args):
             "clocks": clk.summary(),
         }
         if args.cpu_baseline:
-            out["cpu_baseline"] = cpu_baseline(spec, d, lin.export(), budget_s=args.cpu_seconds)
+            out["cpu_baseline"] = cpu_baseline(spec, d, lin.export(), budget_s=args.cpu_seconds,
+                                               fmt=args.format)
         print(json.dumps(out), flush=True)
     if world > 1:
         dist.barrier()
@@ -448,11 +471,25 @@ def _blas_threads():
     return os.cpu_count()
 
 
-def cpu_baseline(spec, d, exp, budget_s=15.0, rows=256):
+class _Int4OracleView:
+    """The INT4 oracle under the NVFP4 oracle's function names used below."""
+
+    def __init__(self, m):
+        self.linear_forward = m.linear_forward_int4
+        self.quantize_act = m.quantize_act_int4
+        self.dequantize = m.dequantize_int4
+
+
+def cpu_baseline(spec, d, exp, budget_s=15.0, rows=256, fmt="nvfp4"):
     """The oracle's forward (activation quantisation, weight dequantisation,
     float64 GEMM, low-rank branch) on a row sample of the workload, repeated
     for about `budget_s` seconds; the weight is the library's exported one."""
-    from oracle import svdq_ref as ref
+    from oracle import int4_ref
+    from oracle import svdq_ref
+    if fmt == "int4":
+        ref = _Int4OracleView(int4_ref)
+    else:
+        ref = svdq_ref
     prep = dict(inv_lambda=exp["inv_lambda"], L1=exp["L1"], L2t=exp["L2t"],
                 w_codes=exp["w_codes"], w_scales=exp["w_scales"], bias=d["bias"])
     X = d["X"][:rows]
@@ -537,6 +574,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--workload", default="qkv")
+    ap.add_argument("--format", choices=["nvfp4", "int4"], default="nvfp4",
+                    help="4-bit format of the layer (int4: the variant for pre-Blackwell checkpoints)")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-rows", type=int, default=128)
@@ -553,6 +592,8 @@ def main(argv=None):
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
         raise SystemExit("for --gpus > 1 launch with torch.distributed.run (one rank per GPU)")
     if args.block:
+        if args.format != "nvfp4":
+            raise SystemExit("--block times the NVFP4 layer")
         return run_block(args)
     return run_native(args)
 

@@ -87,10 +87,24 @@ typedef enum svdq_status {
  *   L2t        N x r bf16, L2^T = V_r.
  *   inv_lambda K float32, f32(1 / lambda).
  *   bias       N bf16, or NULL when has_bias == 0.
+ *
+ * INT4 format (format == SVDQ_FORMAT_INT4): the other 4-bit format of the
+ * layer, used before Blackwell (chaosnode.de "Nunchaku Lite", section
+ * "Hardware-Support").  w_codes has the same N x K/2 shape and nibble order,
+ * the nibbles being two's-complement integers in [-8, 7]; w_scales holds one
+ * fp16 scale per group of 64 elements along K, group-major: fp16 [K/64][N]
+ * (scale of row n, group g at element g * N + n; N * K / 32 bytes, a prefix
+ * of the field).  Quantiser of a group v[64]: s = fp16_RNE(min(f32(max|v| /
+ * 7), 65504)), q = clamp(RNE(f32(v / s)), -8, 7), q = 0 when s == 0.  All
+ * other fields are shared with NVFP4.
  */
+#define SVDQ_FORMAT_NVFP4 0
+#define SVDQ_FORMAT_INT4 1
+
 typedef struct svdq_weight {
   int32_t N, K, r;
   int32_t has_bias;
+  int32_t format;     /* SVDQ_FORMAT_NVFP4 (default of svdq_weight_bind) or SVDQ_FORMAT_INT4 */
   uint8_t* w_codes;
   uint8_t* w_scales;
   uint16_t* L1;
@@ -133,6 +147,12 @@ size_t svdq_prepare_workspace_bytes(int N, int K, int r);
 svdq_status svdq_weight_bind(void* buf, size_t bytes, int N, int K, int r, int has_bias,
                              svdq_weight* out);
 
+/* svdq_weight_bind, then out->format = format (SVDQ_FORMAT_NVFP4 or
+ * SVDQ_FORMAT_INT4; anything else is SVDQ_ERR_INVALID_ARG).  Every entry point
+ * that takes the weight follows its format. */
+svdq_status svdq_weight_bind_format(void* buf, size_t bytes, int N, int K, int r, int has_bias, int format,
+                                    svdq_weight* out);
+
 /* ---------------------------------------------------------------------------
  * Offline preparation (smoothing, rank-r split, residual NVFP4 pack).
  *   W       device, N x K bf16 (nn.Linear weight)
@@ -146,7 +166,7 @@ svdq_status svdq_weight_bind(void* buf, size_t bytes, int N, int K, int r, int h
  * (the smaller of What What^T and What^T What), each pair sign-normalised so
  * the largest-|.| entry of u_i is positive, stored as bf16 (RNE);
  * R = f32(What - (bf16 L1 bf16 L2)^T) summed in float64; R quantised to NVFP4
- * along K.  Offline: it creates (and destroys) one cuSOLVER handle per call,
+ * along K (to INT4 groups of 64 when w->format == SVDQ_FORMAT_INT4).  Offline: it creates (and destroys) one cuSOLVER handle per call,
  * whose own small allocation is the one exception to "never allocates", and
  * the solver may synchronise the stream.
  * ------------------------------------------------------------------------- */
@@ -161,6 +181,9 @@ svdq_status svdq_prepare_weight(const uint16_t* W, const float* lambda, const ui
  *            M .. roundup(M,128)-1 are written as zero
  *   D        device, M x r bf16, D = bf16(sum_k bf16(Xhat)_mk bf16(L1)_kj)
  *            with float32 accumulation; may be NULL when r == 0
+ * With an INT4 weight the codes are INT4 and x_scales holds fp16 group scales
+ * group-major, [K/64][roundup(M,128)] (scale of row m, group g at element
+ * g * roundup(M,128) + m; padding rows zero); the buffer size above covers it.
  * ------------------------------------------------------------------------- */
 svdq_status svdq_quantize_act(const uint16_t* X, int M, const svdq_weight* w, uint8_t* x_codes,
                               uint8_t* x_scales, uint16_t* D, void* stream);
@@ -173,6 +196,10 @@ svdq_status svdq_quantize_act(const uint16_t* X, int M, const svdq_weight* w, ui
  * output tiles (N % 256 == 0 and at least one tile per SM) or 128 x 128 tiles
  * (SVDQ_GEMM_BN=128|256 overrides); with SVDQ_GEMM_PAIR=1 and N % 256 == 0,
  * CTA pairs compute 256 x 256 tiles with two-CTA MMAs instead.
+ * With an INT4 weight: Y = bf16(sum_g sx[m,g] sw[n,g] (sum_{k in group g}
+ * qx[m,k] qw[n,k]) + D L2 + bias), the integer group sums exact (8-bit integer
+ * warp MMA on the sign-extended codes) and the scaling in float32; 128 x 128
+ * tiles, one CTA each.
  * ------------------------------------------------------------------------- */
 svdq_status svdq_gemm(const uint8_t* x_codes, const uint8_t* x_scales, const uint16_t* D, int M,
                       const svdq_weight* w, uint16_t* Y, void* stream);
@@ -289,6 +316,14 @@ svdq_status svdq_calibrate_lambda(const float* x_absmax, const uint16_t* W, int 
  * entries are written as 0 by to_native and ignored by to_logical). */
 svdq_status svdq_scales_to_logical(const uint8_t* native, int rows, int K, uint8_t* logical);
 svdq_status svdq_scales_to_native(const uint8_t* logical, int rows, int K, uint8_t* native);
+
+/* Host-only conversions of INT4 fp16 scales between the logical [rows][K/64]
+ * layout and the group-major [K/64][rows_pad] one (rows_pad >= rows: N for a
+ * weight, roundup(M,128) for activations; padding written as 0). */
+svdq_status svdq_int4_scales_to_logical(const uint16_t* native, int rows, int rows_pad, int K,
+                                        uint16_t* logical);
+svdq_status svdq_int4_scales_to_native(const uint16_t* logical, int rows, int rows_pad, int K,
+                                       uint16_t* native);
 
 /* Synchronise `stream` and report the device status word of the current
  * device: SVDQ_OK, or SVDQ_ERR_TIMEOUT if a kernel gave up a bounded wait

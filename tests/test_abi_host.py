@@ -138,3 +138,42 @@ def svdq_weight_copy(w):
     c = binding.svdq_weight()
     ctypes.memmove(ctypes.byref(c), ctypes.byref(w), ctypes.sizeof(w))
     return c
+
+
+def test_weight_format_field_and_validation():
+    N, K, r = 256, 512, 32
+    nbytes = svdq.svdq_weight_bytes(N, K, r, 1)
+    base = 0x7F0000000000
+    assert svdq.svdq_weight_bind(base, nbytes, N, K, r, 1).format == svdq.SVDQ_FORMAT_NVFP4
+    w4 = svdq.svdq_weight_bind_format(base, nbytes, N, K, r, 1, svdq.SVDQ_FORMAT_INT4)
+    assert w4.format == svdq.SVDQ_FORMAT_INT4
+    # the INT4 scale table (N x K/64 fp16) fits in the field before L1
+    assert w4.w_scales + N * (K // 64) * 2 <= w4.L1
+    with pytest.raises(svdq.SvdqError, match="INVALID_ARG"):
+        svdq.svdq_weight_bind_format(base, nbytes, N, K, r, 1, 7)
+    lib = svdq.lib()
+    A = 0x7E0000000000
+    bad = svdq_weight_copy(w4)
+    bad.format = 3
+    assert lib.svdq_quantize_act(A, 64, ctypes.byref(bad), A, A, A, None) == 1
+    assert lib.svdq_gemm(A, A, A, 64, ctypes.byref(bad), A, None) == 1
+    # the activation scale buffer covers the INT4 group-major table too
+    M = 130
+    assert svdq.svdq_act_scales_bytes(M, K) >= ((M + 127) // 128 * 128) * (K // 64) * 2
+
+
+@pytest.mark.parametrize("rows,rows_pad,K", [(1, 128, 64), (130, 256, 256), (256, 256, 3072)])
+def test_int4_scale_layout_roundtrip(rows, rows_pad, K):
+    """Group-major fp16 layout restated from include/svdq.h: row i, group g at g * rows_pad + i."""
+    rng = np.random.default_rng(rows + K)
+    logical = rng.integers(0, 0x7C00, (rows, K // 64)).astype(np.uint16)
+    native = np.full(rows_pad * (K // 64), 0xAAAA, np.uint16)
+    svdq.svdq_int4_scales_to_native(logical.ctypes.data, rows, rows_pad, K, native.ctypes.data)
+    nat2 = native.reshape(K // 64, rows_pad)
+    assert np.array_equal(nat2[:, :rows].T, logical)
+    assert np.all(nat2[:, rows:] == 0)
+    back = np.empty_like(logical)
+    svdq.svdq_int4_scales_to_logical(native.ctypes.data, rows, rows_pad, K, back.ctypes.data)
+    assert np.array_equal(back, logical)
+    with pytest.raises(svdq.SvdqError, match="INVALID_ARG"):
+        svdq.svdq_int4_scales_to_logical(native.ctypes.data, rows, rows - 1, K, back.ctypes.data)

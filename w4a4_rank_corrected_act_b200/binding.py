@@ -18,6 +18,9 @@ _PKG_DIR = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG_DIR, "libsvdq_b200.so")
 
 SVDQ_OK = 0
+SVDQ_FORMAT_NVFP4 = 0
+SVDQ_FORMAT_INT4 = 1
+FORMAT_NAMES = {"nvfp4": SVDQ_FORMAT_NVFP4, "int4": SVDQ_FORMAT_INT4}
 STATUS_NAMES = {
     0: "SVDQ_OK", 1: "SVDQ_ERR_INVALID_ARG", 2: "SVDQ_ERR_UNSUPPORTED_SHAPE",
     3: "SVDQ_ERR_MISALIGNED", 4: "SVDQ_ERR_WORKSPACE_TOO_SMALL", 5: "SVDQ_ERR_CUDA",
@@ -33,7 +36,7 @@ _SZ = ctypes.c_size_t
 class svdq_weight(ctypes.Structure):
     _fields_ = [
         ("N", ctypes.c_int32), ("K", ctypes.c_int32), ("r", ctypes.c_int32),
-        ("has_bias", ctypes.c_int32),
+        ("has_bias", ctypes.c_int32), ("format", ctypes.c_int32),
         ("w_codes", _P), ("w_scales", _P), ("L1", _P), ("L1f", _P), ("L2t", _P),
         ("inv_lambda", _P), ("bias", _P),
     ]
@@ -51,6 +54,7 @@ SIGNATURES = {
     "svdq_forward_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
     "svdq_prepare_workspace_bytes": (_SZ, [_I, _I, _I]),
     "svdq_weight_bind": (_I, [_P, _SZ, _I, _I, _I, _I, _WP]),
+    "svdq_weight_bind_format": (_I, [_P, _SZ, _I, _I, _I, _I, _I, _WP]),
     "svdq_prepare_weight": (_I, [_P, _P, _P, _WP, _P, _SZ, _P]),
     "svdq_quantize_act": (_I, [_P, _I, _WP, _P, _P, _P, _P]),
     "svdq_gemm": (_I, [_P, _P, _P, _I, _WP, _P, _P]),
@@ -65,6 +69,8 @@ SIGNATURES = {
     "svdq_calibrate_lambda": (_I, [_P, _P, _I, _I, ctypes.c_float, _P, _P]),
     "svdq_scales_to_logical": (_I, [_P, _I, _I, _P]),
     "svdq_scales_to_native": (_I, [_P, _I, _I, _P]),
+    "svdq_int4_scales_to_logical": (_I, [_P, _I, _I, _I, _P]),
+    "svdq_int4_scales_to_native": (_I, [_P, _I, _I, _I, _P]),
     "svdq_get_device_status": (_I, [_P, ctypes.POINTER(ctypes.c_uint32)]),
     "svdq_clear_device_status": (_I, [_P]),
     "svdq_selftest_wait_timeout": (_I, [ctypes.c_uint64, _P]),
@@ -148,6 +154,13 @@ def svdq_weight_bind(buf: int, nbytes: int, N: int, K: int, r: int, has_bias: in
     return w
 
 
+def svdq_weight_bind_format(buf: int, nbytes: int, N: int, K: int, r: int, has_bias: int,
+                            format: int) -> svdq_weight:
+    w = svdq_weight()
+    _call("svdq_weight_bind_format", buf, nbytes, N, K, r, has_bias, format, ctypes.byref(w))
+    return w
+
+
 def svdq_prepare_weight(W: int, lam: int, bias: int, w: svdq_weight, ws: int, ws_bytes: int,
                         stream: int) -> None:
     _call("svdq_prepare_weight", W, lam, bias or None, ctypes.byref(w), ws, ws_bytes, stream or None)
@@ -223,6 +236,14 @@ def svdq_scales_to_native(logical: int, rows: int, K: int, native: int) -> None:
     _call("svdq_scales_to_native", logical, rows, K, native)
 
 
+def svdq_int4_scales_to_logical(native: int, rows: int, rows_pad: int, K: int, logical: int) -> None:
+    _call("svdq_int4_scales_to_logical", native, rows, rows_pad, K, logical)
+
+
+def svdq_int4_scales_to_native(logical: int, rows: int, rows_pad: int, K: int, native: int) -> None:
+    _call("svdq_int4_scales_to_native", logical, rows, rows_pad, K, native)
+
+
 def svdq_get_device_status(stream: int = 0) -> int:
     """Returns the raw device status word (0 = no kernel gave up a wait)."""
     detail = ctypes.c_uint32(0)
@@ -267,18 +288,23 @@ def _stream_handle(stream=None) -> int:
     return int(s.cuda_stream)
 
 
+# weight-file format tags written by SvdqLinear.save
+_FILE_FORMATS = {"nvfp4": "svdq-w4a4-nvfp4-1", "int4": "svdq-w4a4-int4-1"}
+
+
 class SvdqLinear:
     """A prepared SVDQuant W4A4 linear on the current CUDA device.
 
     ``W`` (N x K), ``lam`` (K, float32) and ``bias`` (N or None) are device
     tensors; the weight is prepared once with ``svdq_prepare_weight`` and kept
-    in one torch-allocated buffer bound with ``svdq_weight_bind``.
+    in one torch-allocated buffer bound with ``svdq_weight_bind_format``.
+    ``format`` is "nvfp4" (the Blackwell format, default) or "int4".
     """
 
-    def __init__(self, W, lam, bias=None, r: int = 32, stream=None):
+    def __init__(self, W, lam, bias=None, r: int = 32, stream=None, format: str = "nvfp4"):
         import torch
         N, K = W.shape
-        self._bind(int(N), int(K), int(r), bias is not None, W.device)
+        self._bind(int(N), int(K), int(r), bias is not None, W.device, format)
         ws_bytes = svdq_prepare_workspace_bytes(self.N, self.K, self.r)
         ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=W.device)
         Wc = W.contiguous()
@@ -289,29 +315,32 @@ class SvdqLinear:
         torch.cuda.current_stream().synchronize() if stream is None else stream.synchronize()
         del ws
 
-    def _bind(self, N: int, K: int, r: int, has_bias: bool, device) -> None:
+    def _bind(self, N: int, K: int, r: int, has_bias: bool, device, format: str = "nvfp4") -> None:
         import torch
+        if format not in FORMAT_NAMES:
+            raise ValueError(f"format must be one of {sorted(FORMAT_NAMES)}")
         self.N, self.K, self.r = N, K, r
         self.has_bias = has_bias
+        self.format = format
         nbytes = svdq_weight_bytes(self.N, self.K, self.r, int(self.has_bias))
         if nbytes == 0:
             raise SvdqError("svdq_weight_bytes", 2, f"N={N} K={K} r={r}")
         self.buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
-        self.w = svdq_weight_bind(self.buf.data_ptr(), nbytes, self.N, self.K, self.r,
-                                  int(self.has_bias))
+        self.w = svdq_weight_bind_format(self.buf.data_ptr(), nbytes, self.N, self.K, self.r,
+                                         int(self.has_bias), FORMAT_NAMES[format])
 
     @classmethod
-    def from_export(cls, exp: dict, bias=None, device="cuda", stream=None):
+    def from_export(cls, exp: dict, bias=None, device="cuda", stream=None, format: str = "nvfp4"):
         """A layer from host arrays in the layouts of ``export()`` (bias: N uint16
         bf16 bits or None), loaded with ``svdq_weight_import``."""
         import numpy as np
         self = cls.__new__(cls)
         N, K2 = exp["w_codes"].shape
         r = int(exp["L1"].shape[1]) if exp.get("L1") is not None else 0
-        self._bind(int(N), int(K2) * 2, r, bias is not None, device)
+        self._bind(int(N), int(K2) * 2, r, bias is not None, device, format)
         # every host array stays referenced until the (synchronous) import returns
         codes = np.ascontiguousarray(exp["w_codes"], dtype=np.uint8)
-        scales = np.ascontiguousarray(exp["w_scales"], dtype=np.uint8)
+        scales = np.ascontiguousarray(exp["w_scales"], dtype=np.uint16 if format == "int4" else np.uint8)
         L1 = np.ascontiguousarray(exp["L1"], dtype=np.uint16) if r else None
         L2t = np.ascontiguousarray(exp["L2t"], dtype=np.uint16) if r else None
         inv = np.ascontiguousarray(exp["inv_lambda"], dtype=np.float32)
@@ -333,18 +362,19 @@ class SvdqLinear:
         import numpy as np
         exp = self.export()
         extra = {"bias": self.bias_host()} if self.has_bias else {}
-        np.savez(path, format=np.array("svdq-w4a4-nvfp4-1"), N=self.N, K=self.K, r=self.r, **exp, **extra)
+        np.savez(path, format=np.array(_FILE_FORMATS[self.format]), N=self.N, K=self.K, r=self.r, **exp, **extra)
 
     @classmethod
     def load(cls, path, device="cuda", stream=None):
         """A layer from a file written by ``save``."""
         import numpy as np
         with np.load(path) as z:
-            if str(z["format"]) != "svdq-w4a4-nvfp4-1":
+            fmt = {v: k for k, v in _FILE_FORMATS.items()}.get(str(z["format"]))
+            if fmt is None:
                 raise ValueError(f"{path}: not an SVDQuant weight file")
             exp = {k: z[k] for k in ("w_codes", "w_scales", "L1", "L2t", "inv_lambda")}
             bias = z["bias"] if "bias" in z.files else None
-        return cls.from_export(exp, bias=bias, device=device, stream=stream)
+        return cls.from_export(exp, bias=bias, device=device, stream=stream, format=fmt)
 
     def workspace_bytes(self, M: int) -> int:
         return svdq_forward_workspace_bytes(M, self.N, self.K, self.r)
@@ -365,7 +395,10 @@ class SvdqLinear:
         """Host copies of the prepared weight in logical layouts (numpy arrays)."""
         import numpy as np
         codes = np.empty((self.N, self.K // 2), np.uint8)
-        scales = np.empty((self.N, self.K // 16), np.uint8)
+        if self.format == "int4":
+            scales = np.empty((self.N, self.K // 64), np.uint16)     # fp16 bits
+        else:
+            scales = np.empty((self.N, self.K // 16), np.uint8)      # E4M3 codes
         L1 = np.empty((self.K, self.r), np.uint16)
         L2t = np.empty((self.N, self.r), np.uint16)
         inv = np.empty(self.K, np.float32)

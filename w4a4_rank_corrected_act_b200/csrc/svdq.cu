@@ -26,6 +26,7 @@
 #include "act_quant.cuh"
 #include "fp4_gemm.cuh"
 #include "fp4_gemm_pair.cuh"
+#include "int4.cuh"
 #include "prepare.cuh"
 
 using namespace svdq;
@@ -68,6 +69,7 @@ svdq_status check_layer_shape(int N, int K, int r) {
 
 svdq_status check_weight(const svdq_weight* w) {
   if (w == nullptr) return SVDQ_ERR_INVALID_ARG;
+  if (w->format != SVDQ_FORMAT_NVFP4 && w->format != SVDQ_FORMAT_INT4) return SVDQ_ERR_INVALID_ARG;
   svdq_status s = check_layer_shape(w->N, w->K, w->r);
   if (s != SVDQ_OK) return s;
   if (w->w_codes == nullptr || w->w_scales == nullptr || w->inv_lambda == nullptr)
@@ -264,8 +266,112 @@ svdq_status dispatch_gemm_r(int r_pad, const CUtensorMap& ta, const CUtensorMap&
   }
 }
 
+// ---- INT4 variant -------------------------------------------------------
+template <int R_PAD>
+svdq_status launch_act_int4(const CUtensorMap& tx, const Int4ActParams& p, cudaStream_t st) {
+  constexpr uint32_t smem = Int4ActSmem<R_PAD>::kBytes;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(act_quant_int4_kernel<R_PAD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    smem);
+  });
+  if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(act int4)");
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(p.M_pad / ACT_ROWS));
+  cfg.blockDim = dim3(ACT_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, act_quant_int4_kernel<R_PAD>, tx, p);
+  if (e != cudaSuccess) return cuda_fail(e, "act_quant_int4_kernel launch");
+  SVDQ_CHECK_LAUNCH("act_quant_int4_kernel");
+  return SVDQ_OK;
+}
+
+svdq_status quantize_act_int4_impl(const uint16_t* X, int M, const svdq_weight* w, uint8_t* x_codes,
+                                   uint8_t* x_scales, uint16_t* D, cudaStream_t st) {
+  const int K = w->K, r = w->r;
+  CUtensorMap tx{};
+  svdq_status s = make_tmap(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M,
+                            static_cast<uint64_t>(K) * 2, ACT_SUB, ACT_ROWS,
+                            CU_TENSOR_MAP_SWIZZLE_128B);
+  if (s != SVDQ_OK) return s;
+  Int4ActParams p;
+  p.inv_lambda = w->inv_lambda;
+  p.L1f = reinterpret_cast<const uint32_t*>(w->L1f);
+  p.x_codes = x_codes;
+  p.x_scales = reinterpret_cast<uint16_t*>(x_scales);
+  p.D = D;
+  p.M = M;
+  p.K = K;
+  p.r = r;
+  p.M_pad = m_pad_of(M);
+  switch (r_pad_of(r)) {
+    case 0: return launch_act_int4<0>(tx, p, st);
+    case 16: return launch_act_int4<16>(tx, p, st);
+    case 32: return launch_act_int4<32>(tx, p, st);
+    default: return launch_act_int4<64>(tx, p, st);
+  }
+}
+
+template <int R_PAD>
+svdq_status launch_gemm_int4(const CUtensorMap* maps, const Int4GemmParams& p, cudaStream_t st) {
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(int4_gemm_kernel<R_PAD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    I4_SMEM_BYTES);
+  });
+  if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(gemm int4)");
+  const dim3 grid(static_cast<unsigned>((p.M + I4_BM - 1) / I4_BM), static_cast<unsigned>(p.N / I4_BN));
+  int4_gemm_kernel<R_PAD><<<grid, I4_THREADS, I4_SMEM_BYTES, st>>>(maps[0], maps[1], maps[2], maps[3], p);
+  SVDQ_CHECK_LAUNCH("int4_gemm_kernel");
+  return SVDQ_OK;
+}
+
+svdq_status gemm_int4_impl(const uint8_t* x_codes, const uint8_t* x_scales, const uint16_t* D, int M,
+                           const svdq_weight* w, uint16_t* Y, cudaStream_t st, int head_dim) {
+  const int N = w->N, K = w->K;
+  const int m_pad = m_pad_of(M);
+  CUtensorMap maps[4] = {};
+  svdq_status s = make_tmap(&maps[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, x_codes, K / 2, M, K / 2, 128, I4_BM,
+                            CU_TENSOR_MAP_SWIZZLE_128B);
+  if (s != SVDQ_OK) return s;
+  s = make_tmap(&maps[1], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->w_codes, K / 2, N, K / 2, 128, I4_BN,
+                CU_TENSOR_MAP_SWIZZLE_128B);
+  if (s != SVDQ_OK) return s;
+  s = make_tmap(&maps[2], CU_TENSOR_MAP_DATA_TYPE_UINT16, x_scales, m_pad, K / INT4_GROUP,
+                static_cast<uint64_t>(m_pad) * 2, I4_BM, I4_GPS, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (s != SVDQ_OK) return s;
+  s = make_tmap(&maps[3], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->w_scales, N, K / INT4_GROUP,
+                static_cast<uint64_t>(N) * 2, I4_BN, I4_GPS, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (s != SVDQ_OK) return s;
+  Int4GemmParams p;
+  p.D = D;
+  p.L2t = w->L2t;
+  p.bias = w->has_bias ? w->bias : nullptr;
+  p.Y = Y;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.r = w->r;
+  p.head_dim = head_dim;
+  switch (r_pad_of(w->r)) {
+    case 0: return launch_gemm_int4<0>(maps, p, st);
+    case 16: return launch_gemm_int4<16>(maps, p, st);
+    case 32: return launch_gemm_int4<32>(maps, p, st);
+    default: return launch_gemm_int4<64>(maps, p, st);
+  }
+}
+
 svdq_status quantize_act_impl(const uint16_t* X, int M, const svdq_weight* w, uint8_t* x_codes,
                               uint8_t* x_scales, uint16_t* D, cudaStream_t st) {
+  if (w->format == SVDQ_FORMAT_INT4) return quantize_act_int4_impl(X, M, w, x_codes, x_scales, D, st);
   const int K = w->K, r = w->r, rp = r_pad_of(r);
   CUtensorMap tx{};
   svdq_status s = make_tmap(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M,
@@ -359,6 +465,7 @@ svdq_status gemm_pair_impl(const uint8_t* x_codes, const uint8_t* x_scales, cons
 // head_dim == 0: Y row-major M x N; else Y head-major [N / head_dim][M][head_dim]
 svdq_status gemm_impl(const uint8_t* x_codes, const uint8_t* x_scales, const uint16_t* D, int M,
                       const svdq_weight* w, uint16_t* Y, cudaStream_t st, int head_dim = 0) {
+  if (w->format == SVDQ_FORMAT_INT4) return gemm_int4_impl(x_codes, x_scales, D, M, w, Y, st, head_dim);
   if (head_dim == 0) {
     // the CTA-pair kernel (256 x 256 tiles) is used on request (SVDQ_GEMM_PAIR=1)
     bool pair = false;
@@ -452,6 +559,7 @@ size_t weight_layout(int N, int K, int r, int has_bias, uint8_t* base, svdq_weig
     out->K = K;
     out->r = r;
     out->has_bias = has_bias ? 1 : 0;
+    out->format = SVDQ_FORMAT_NVFP4;
     out->w_codes = codes;
     out->w_scales = scales;
     out->L1 = r > 0 ? reinterpret_cast<uint16_t*>(l1) : nullptr;
@@ -522,6 +630,22 @@ void to_logical(const uint8_t* native, int rows, int K, uint8_t* logical) {
   for (int i = 0; i < rows; ++i)
     for (int j = 0; j < kb; ++j)
       logical[static_cast<size_t>(i) * kb + j] = native[sf_offset(i, j, K)];
+}
+
+// INT4 scales: native fp16 [K/64][rows_pad] (group-major) <-> logical [rows][K/64].
+void int4_to_logical(const uint16_t* native, int rows, int rows_pad, int K, uint16_t* logical) {
+  const int ng = K / INT4_GROUP;
+  for (int i = 0; i < rows; ++i)
+    for (int g = 0; g < ng; ++g)
+      logical[static_cast<size_t>(i) * ng + g] = native[static_cast<size_t>(g) * rows_pad + i];
+}
+
+void int4_to_native(const uint16_t* logical, int rows, int rows_pad, int K, uint16_t* native) {
+  const int ng = K / INT4_GROUP;
+  std::memset(native, 0, static_cast<size_t>(rows_pad) * ng * 2);
+  for (int i = 0; i < rows; ++i)
+    for (int g = 0; g < ng; ++g)
+      native[static_cast<size_t>(g) * rows_pad + i] = logical[static_cast<size_t>(i) * ng + g];
 }
 
 // One bounded wait on an mbarrier that nothing arrives on: the same wait the
@@ -743,6 +867,14 @@ svdq_status svdq_weight_bind(void* buf, size_t bytes, int N, int K, int r, int h
   return SVDQ_OK;
 }
 
+svdq_status svdq_weight_bind_format(void* buf, size_t bytes, int N, int K, int r, int has_bias, int format,
+                                    svdq_weight* out) {
+  if (format != SVDQ_FORMAT_NVFP4 && format != SVDQ_FORMAT_INT4) return SVDQ_ERR_INVALID_ARG;
+  const svdq_status s = svdq_weight_bind(buf, bytes, N, K, r, has_bias, out);
+  if (s == SVDQ_OK) out->format = format;
+  return s;
+}
+
 svdq_status svdq_prepare_weight(const uint16_t* W, const float* lambda, const uint16_t* bias,
                                 const svdq_weight* w, void* ws, size_t ws_bytes, void* stream) {
   svdq_status s = check_weight(w);
@@ -817,7 +949,15 @@ svdq_status svdq_prepare_weight(const uint16_t* W, const float* lambda, const ui
     e = cudaGetLastError();
     if (e != cudaSuccess) return fail(cuda_fail(e, "prepare factor kernels"));
   }
-  switch (r_pad_of(r)) {
+  uint16_t* s16 = reinterpret_cast<uint16_t*>(w->w_scales);
+  if (w->format == SVDQ_FORMAT_INT4) {
+    switch (r_pad_of(r)) {
+      case 0: prep_residual_int4_kernel<0><<<N, 256, 0, st>>>(pw.what, w->L1, w->L2t, N, K, r, w->w_codes, s16); break;
+      case 16: prep_residual_int4_kernel<16><<<N, 256, 0, st>>>(pw.what, w->L1, w->L2t, N, K, r, w->w_codes, s16); break;
+      case 32: prep_residual_int4_kernel<32><<<N, 256, 0, st>>>(pw.what, w->L1, w->L2t, N, K, r, w->w_codes, s16); break;
+      default: prep_residual_int4_kernel<64><<<N, 256, 0, st>>>(pw.what, w->L1, w->L2t, N, K, r, w->w_codes, s16); break;
+    }
+  } else switch (r_pad_of(r)) {
     case 0: prep_residual_kernel<0><<<N, 256, 0, st>>>(pw.what, w->L1, w->L2t, N, K, r, w->w_codes, w->w_scales); break;
     case 16: prep_residual_kernel<16><<<N, 256, 0, st>>>(pw.what, w->L1, w->L2t, N, K, r, w->w_codes, w->w_scales); break;
     case 32: prep_residual_kernel<32><<<N, 256, 0, st>>>(pw.what, w->L1, w->L2t, N, K, r, w->w_codes, w->w_scales); break;
@@ -1008,10 +1148,11 @@ svdq_status svdq_weight_export(const svdq_weight* w, uint8_t* host_codes, uint8_
   if (s != SVDQ_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t N = w->N, K = w->K, r = w->r;
+  const bool int4 = w->format == SVDQ_FORMAT_INT4;
   std::vector<uint8_t> native;
   if (host_codes) SVDQ_CUDA(cudaMemcpyAsync(host_codes, w->w_codes, N * K / 2, cudaMemcpyDeviceToHost, st));
   if (host_scales) {
-    native.resize(N * K / 16);
+    native.resize(int4 ? N * K / 32 : N * K / 16);
     SVDQ_CUDA(cudaMemcpyAsync(native.data(), w->w_scales, native.size(), cudaMemcpyDeviceToHost, st));
   }
   if (host_L1 && r) SVDQ_CUDA(cudaMemcpyAsync(host_L1, w->L1, K * r * 2, cudaMemcpyDeviceToHost, st));
@@ -1019,7 +1160,13 @@ svdq_status svdq_weight_export(const svdq_weight* w, uint8_t* host_codes, uint8_
   if (host_inv_lambda)
     SVDQ_CUDA(cudaMemcpyAsync(host_inv_lambda, w->inv_lambda, K * 4, cudaMemcpyDeviceToHost, st));
   SVDQ_CUDA(cudaStreamSynchronize(st));
-  if (host_scales) to_logical(native.data(), w->N, w->K, host_scales);
+  if (host_scales) {
+    if (int4)
+      int4_to_logical(reinterpret_cast<const uint16_t*>(native.data()), w->N, w->N, w->K,
+                      reinterpret_cast<uint16_t*>(host_scales));
+    else
+      to_logical(native.data(), w->N, w->K, host_scales);
+  }
   return SVDQ_OK;
 }
 
@@ -1033,8 +1180,12 @@ svdq_status svdq_weight_import(const svdq_weight* w, const uint8_t* host_codes, 
     return SVDQ_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t N = w->N, K = w->K, r = w->r;
-  std::vector<uint8_t> native(N * K / 16);
-  to_native(host_scales, w->N, w->K, native.data());
+  std::vector<uint8_t> native(w->format == SVDQ_FORMAT_INT4 ? N * K / 32 : N * K / 16);
+  if (w->format == SVDQ_FORMAT_INT4)
+    int4_to_native(reinterpret_cast<const uint16_t*>(host_scales), w->N, w->N, w->K,
+                   reinterpret_cast<uint16_t*>(native.data()));
+  else
+    to_native(host_scales, w->N, w->K, native.data());
   SVDQ_CUDA(cudaMemcpyAsync(w->w_codes, host_codes, N * K / 2, cudaMemcpyHostToDevice, st));
   SVDQ_CUDA(cudaMemcpyAsync(w->w_scales, native.data(), native.size(), cudaMemcpyHostToDevice, st));
   if (r) {
@@ -1073,6 +1224,22 @@ svdq_status svdq_calibrate_lambda(const float* x_absmax, const uint16_t* W, int 
   SVDQ_CHECK_LAUNCH("calib_absmax_kernel");
   calib_lambda_kernel<<<(K + 255) / 256, 256, 0, st>>>(x_absmax, K, static_cast<double>(alpha), lambda);
   SVDQ_CHECK_LAUNCH("calib_lambda_kernel");
+  return SVDQ_OK;
+}
+
+svdq_status svdq_int4_scales_to_logical(const uint16_t* native, int rows, int rows_pad, int K,
+                                        uint16_t* logical) {
+  if (native == nullptr || logical == nullptr || rows < 0 || rows_pad < rows || K <= 0 || K % INT4_GROUP)
+    return SVDQ_ERR_INVALID_ARG;
+  int4_to_logical(native, rows, rows_pad, K, logical);
+  return SVDQ_OK;
+}
+
+svdq_status svdq_int4_scales_to_native(const uint16_t* logical, int rows, int rows_pad, int K,
+                                       uint16_t* native) {
+  if (native == nullptr || logical == nullptr || rows < 0 || rows_pad < rows || K <= 0 || K % INT4_GROUP)
+    return SVDQ_ERR_INVALID_ARG;
+  int4_to_native(logical, rows, rows_pad, K, native);
   return SVDQ_OK;
 }
 
