@@ -41,10 +41,15 @@
  *   - Errors are returned as status codes; nothing is thrown across the ABI.
  *     A CUDA launch/runtime failure is SVDQ_ERR_CUDA (its text is kept in a
  *     thread-local string, see svdq_last_error_detail).
- *   - The library is stateless apart from a per-device status word that
- *     kernels set when a bounded wait times out (svdq_get_device_status):
- *     bit 0 = timeout, bits 8-15 = kernel (1 activation, 2 GEMM, 3 prepare,
- *     4 self-test), bits 16-23 = wait site.  Every wait gives up after 1 s.
+ *   - The library keeps no state between calls apart from a per-device status
+ *     word that kernels set when a bounded wait times out
+ *     (svdq_get_device_status): bit 0 = timeout, bits 8-15 = kernel
+ *     (1 activation, 2 GEMM, 3 prepare, 4 self-test, 5 INT4 kernels), bits
+ *     16-23 = wait site.  Every wait gives up after 1 s.  Two entry points
+ *     also own per-device resources created on first use: the copy-out stream
+ *     and events of svdq_linear_forward_host (concurrent callers on one device
+ *     enqueue one after the other) and the scratch of
+ *     svdq_linear_forward_noalloc.
  */
 #ifndef SVDQ_H_
 #define SVDQ_H_
@@ -316,6 +321,11 @@ svdq_status svdq_calibrate_lambda(const float* x_absmax, const uint16_t* W, int 
  * entries are written as 0 by to_native and ignored by to_logical). */
 svdq_status svdq_scales_to_logical(const uint8_t* native, int rows, int K, uint8_t* logical);
 svdq_status svdq_scales_to_native(const uint8_t* logical, int rows, int K, uint8_t* native);
+
+/* The activation scales of svdq_quantize_act (M token rows) in logical
+ * [M][K/16] order: svdq_scales_to_logical under the name the interface's
+ * checkpoint/test tooling uses. */
+svdq_status svdq_act_scales_to_logical(const uint8_t* native, int M, int K, uint8_t* logical);
 
 /* Host-only conversions of INT4 fp16 scales between the logical [rows][K/64]
  * layout and the group-major [K/64][rows_pad] one (rows_pad >= rows: N for a

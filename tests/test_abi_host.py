@@ -177,3 +177,14 @@ def test_int4_scale_layout_roundtrip(rows, rows_pad, K):
     assert np.array_equal(back, logical)
     with pytest.raises(svdq.SvdqError, match="INVALID_ARG"):
         svdq.svdq_int4_scales_to_logical(native.ctypes.data, rows, rows - 1, K, back.ctypes.data)
+
+
+def test_act_scales_to_logical_is_the_same_conversion():
+    rows, K = 130, 256
+    rng = np.random.default_rng(3)
+    logical = rng.integers(0, 0x7F, (rows, K // 16)).astype(np.uint8)
+    native = np.zeros(((rows + 127) // 128 * 128) * (K // 16), np.uint8)
+    svdq.svdq_scales_to_native(logical.ctypes.data, rows, K, native.ctypes.data)
+    a = np.empty_like(logical)
+    svdq.svdq_act_scales_to_logical(native.ctypes.data, rows, K, a.ctypes.data)
+    assert np.array_equal(a, logical)

@@ -69,6 +69,7 @@ SIGNATURES = {
     "svdq_calibrate_lambda": (_I, [_P, _P, _I, _I, ctypes.c_float, _P, _P]),
     "svdq_scales_to_logical": (_I, [_P, _I, _I, _P]),
     "svdq_scales_to_native": (_I, [_P, _I, _I, _P]),
+    "svdq_act_scales_to_logical": (_I, [_P, _I, _I, _P]),
     "svdq_int4_scales_to_logical": (_I, [_P, _I, _I, _I, _P]),
     "svdq_int4_scales_to_native": (_I, [_P, _I, _I, _I, _P]),
     "svdq_get_device_status": (_I, [_P, ctypes.POINTER(ctypes.c_uint32)]),
@@ -230,6 +231,10 @@ def svdq_calibrate_lambda(x_absmax: int, W: int, N: int, K: int, alpha: float, l
 
 def svdq_scales_to_logical(native: int, rows: int, K: int, logical: int) -> None:
     _call("svdq_scales_to_logical", native, rows, K, logical)
+
+
+def svdq_act_scales_to_logical(native: int, M: int, K: int, logical: int) -> None:
+    _call("svdq_act_scales_to_logical", native, M, K, logical)
 
 
 def svdq_scales_to_native(logical: int, rows: int, K: int, native: int) -> None:

@@ -1045,6 +1045,7 @@ svdq_status svdq_linear_forward_heads(const uint16_t* X, int M, const svdq_weigh
 // Copy-out stream and events of the host-buffer path, created once per device.
 struct HostPipe {
   static constexpr int kEvents = 8;
+  std::mutex mu;               // one caller at a time enqueues through the pipe
   cudaStream_t out = nullptr;
   cudaEvent_t ev[kEvents] = {};
   cudaEvent_t done = nullptr;
@@ -1097,6 +1098,9 @@ svdq_status svdq_linear_forward_host(const uint16_t* X_host, int M, const svdq_w
   HostPipe* hp = nullptr;
   s = host_pipe(&hp);
   if (s != SVDQ_OK) return s;
+  // the events and the copy-out stream are shared by every caller on this
+  // device: concurrent callers enqueue one after the other
+  std::lock_guard<std::mutex> pipe_lock(hp->mu);
   int i = 0;
   for (int r0 = 0; r0 < M; r0 += kChunk, ++i) {
     const int rows = std::min(kChunk, M - r0);
@@ -1247,6 +1251,10 @@ svdq_status svdq_scales_to_logical(const uint8_t* native, int rows, int K, uint8
   if (native == nullptr || logical == nullptr || rows < 0 || K <= 0 || K % 64) return SVDQ_ERR_INVALID_ARG;
   to_logical(native, rows, K, logical);
   return SVDQ_OK;
+}
+
+svdq_status svdq_act_scales_to_logical(const uint8_t* native, int M, int K, uint8_t* logical) {
+  return svdq_scales_to_logical(native, M, K, logical);
 }
 
 svdq_status svdq_scales_to_native(const uint8_t* logical, int rows, int K, uint8_t* native) {
