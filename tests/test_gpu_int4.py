@@ -227,7 +227,8 @@ def test_int4_export_import_and_file_round_trip(tmp_path):
     lin, exp = _prepare(W, lam, B, r)
     Xd = dev_u16(X).view(t.bfloat16)
     Y0 = lin.forward(Xd)
-    lin2 = svdq.SvdqLinear.from_export(exp, bias=B, format="int4")
+    lin2 = svdq.SvdqLinear.from_export(exp, bias=B)       # format implied by the fp16 scales
+    assert lin2.format == "int4"
     path = tmp_path / "w_int4.npz"
     lin.save(path)
     lin3 = svdq.SvdqLinear.load(path)

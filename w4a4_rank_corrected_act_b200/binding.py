@@ -335,10 +335,14 @@ class SvdqLinear:
                                          int(self.has_bias), FORMAT_NAMES[format])
 
     @classmethod
-    def from_export(cls, exp: dict, bias=None, device="cuda", stream=None, format: str = "nvfp4"):
+    def from_export(cls, exp: dict, bias=None, device="cuda", stream=None, format: Optional[str] = None):
         """A layer from host arrays in the layouts of ``export()`` (bias: N uint16
-        bf16 bits or None), loaded with ``svdq_weight_import``."""
+        bf16 bits or None), loaded with ``svdq_weight_import``.  ``format`` defaults
+        to the one the scales imply: fp16 group scales (uint16) are INT4, E4M3
+        codes (uint8) NVFP4."""
         import numpy as np
+        if format is None:
+            format = "int4" if np.asarray(exp["w_scales"]).dtype == np.uint16 else "nvfp4"
         self = cls.__new__(cls)
         N, K2 = exp["w_codes"].shape
         r = int(exp["L1"].shape[1]) if exp.get("L1") is not None else 0
