@@ -265,3 +265,30 @@ def test_int4_full_size_sampled():
     extra = d_propagated_bound(o["D"], o["D_abs"], exp["L2t"])
     check_y(to_np_u16(Y.view(t.int16))[rows], o["Y64"], "int4 qkv", extra=extra)
     assert svdq.svdq_get_device_status(stream()) == 0
+
+
+@pytest.mark.parametrize("M", [200, 2600])
+def test_int4_host_buffers_and_noalloc_match_device_path(M):
+    """The host-buffer path (chunked above 1024 rows) and the no-allocation path
+    run the same INT4 kernels: their outputs equal the workspace path's bit for bit."""
+    t = torch()
+    K, N, r = 512, 384, 32
+    X, W, B, lam = _inputs(M, K, N, seed=95)
+    lin, _ = _prepare(W, lam, B, r)
+    Yd = to_np_u16(lin.forward(dev_u16(X).view(t.bfloat16)).view(t.int16))
+    Xh = t.from_numpy(X.view(np.int16).copy()).pin_memory()
+    Yh = t.empty((M, N), dtype=t.int16).pin_memory()
+    Xdev = t.empty((M, K), dtype=t.int16, device="cuda")
+    Ydev = t.empty((M, N), dtype=t.int16, device="cuda")
+    nb = lin.workspace_bytes(M)
+    ws = empty_u8(nb)
+    t.cuda.synchronize()
+    svdq.svdq_linear_forward_host(Xh.data_ptr(), M, lin.w, Yh.data_ptr(), Xdev.data_ptr(),
+                                  Ydev.data_ptr(), ws.data_ptr(), nb, stream())
+    t.cuda.current_stream().synchronize()
+    assert np.array_equal(Yh.numpy().view(np.uint16), Yd)
+    Xd = dev_u16(X)
+    Yn = t.full((M, N), -1, dtype=t.int16, device="cuda")
+    svdq.svdq_linear_forward_noalloc(Xd.data_ptr(), M, lin.w, Yn.data_ptr(), stream())
+    t.cuda.synchronize()
+    assert np.array_equal(to_np_u16(Yn), Yd)

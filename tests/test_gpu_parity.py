@@ -345,6 +345,47 @@ def test_forward_host_buffers_match_device_path(M):
     assert np.array_equal(Yh.numpy().view(np.uint16), Yd)
 
 
+def test_forward_host_buffers_concurrent_callers():
+    """Two host threads drive the pipelined host-buffer path at the same time on
+    their own streams (the copy-out stream and events are shared per device):
+    each result must equal its device-path result."""
+    import threading
+    t = torch()
+    M, K, N, r = 2600, 512, 384, 32
+    runs = []
+    for seed in (92, 93):
+        X, W, B, lam = _inputs(M, K, N, seed=seed)
+        lin, _ = _prepare(W, lam, B, r)
+        Yd = to_np_u16(lin.forward(dev_u16(X).view(t.bfloat16)).view(t.int16))
+        nb = lin.workspace_bytes(M)
+        runs.append(dict(lin=lin, Yd=Yd, nb=nb, ws=empty_u8(nb), st=t.cuda.Stream(),
+                         Xh=t.from_numpy(X.view(np.int16).copy()).pin_memory(),
+                         Yh=t.empty((M, N), dtype=t.int16).pin_memory(),
+                         Xdev=t.empty((M, K), dtype=t.int16, device="cuda"),
+                         Ydev=t.empty((M, N), dtype=t.int16, device="cuda")))
+    t.cuda.synchronize()
+    errors = []
+
+    def drive(rr):
+        try:
+            for _ in range(3):
+                svdq.svdq_linear_forward_host(rr["Xh"].data_ptr(), M, rr["lin"].w, rr["Yh"].data_ptr(),
+                                              rr["Xdev"].data_ptr(), rr["Ydev"].data_ptr(),
+                                              rr["ws"].data_ptr(), rr["nb"], int(rr["st"].cuda_stream))
+        except Exception as e:   # reported on the main thread
+            errors.append(e)
+
+    threads = [threading.Thread(target=drive, args=(rr,)) for rr in runs]
+    for th in threads:
+        th.start()
+    for th in threads:
+        th.join()
+    assert not errors, errors
+    for rr in runs:
+        rr["st"].synchronize()
+        assert np.array_equal(rr["Yh"].numpy().view(np.uint16), rr["Yd"])
+
+
 def test_empty_and_invalid_calls():
     t = torch()
     M, K, N, r = 64, 256, 128, 16
