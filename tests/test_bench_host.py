@@ -1,0 +1,65 @@
+"""Host logic of bench.py on CPU: the staleness rule of the committed ncu
+traffic figures, the CPU-baseline leg for both 4-bit formats, and the JSON
+contract of the reference arm (the CPU oracle) on the smallest workload."""
+import json
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from oracle import int4_ref  # noqa: E402
+from oracle import svdq_ref as ref  # noqa: E402
+from workloads import gen  # noqa: E402
+
+
+def test_profile_traffic_only_for_the_profiled_source(tmp_path, monkeypatch):
+    src = tmp_path / "kernel.cuh"
+    src.write_text("// kernel v1\n")
+    (tmp_path / "profiles").mkdir()
+    sha = bench._src_sha([str(src)])
+    (tmp_path / "profiles" / "k_w.txt").write_text(
+        f"header\ncommand: x\nsource_sha: {sha}\ntraffic_bytes_per_launch: 12345\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench._profile_traffic([str(src)], "k_w.txt") == 12345.0
+    assert bench._profile_traffic([str(src)], "missing.txt") is None
+    src.write_text("// kernel v2\n")                        # the kernel changed since the capture
+    assert bench._profile_traffic([str(src)], "k_w.txt") is None
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4"])
+def test_cpu_baseline_leg(fmt):
+    spec = gen.workload("small")
+    d = gen.make_linear(spec)
+    if fmt == "int4":
+        prep = int4_ref.prepare_weight_int4(d["W"], d["lam"], d["bias"], spec.r)
+    else:
+        prep = ref.prepare_weight(d["W"], d["lam"], d["bias"], spec.r)
+    exp = {k: prep[k] for k in ("w_codes", "w_scales", "L1", "L2t", "inv_lambda")}
+    out = bench.cpu_baseline(spec, d, exp, budget_s=0.05, rows=8, fmt=fmt)
+    assert out["kind"] == "oracle" and out["unit"] == bench.UNIT
+    assert out["value"] > 0 and out["cores"] >= 1
+    assert "8 of 256 token rows" in out["sample"]
+
+
+def test_reference_arm_json_line(capsys):
+    out = bench.main(["--impl", "reference", "--workload", "small", "--steps", "1", "--warmup", "3",
+                      "--ref-rows", "8"])
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line == json.loads(json.dumps(out))
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e", "gpu_launches"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+    assert line["cpu_baseline"]["value"] == line["value"]
+    assert line["config"]["workload"].startswith("small")
+
+
+def test_warmup_below_three_is_refused():
+    with pytest.raises(SystemExit):
+        bench.main(["--impl", "reference", "--workload", "small", "--warmup", "2"])
