@@ -18,9 +18,9 @@
 // B200 has no 4-bit integer tensor-core MMA and tcgen05 has no per-group
 // scaling for integers, so the GEMM runs the exact integer group sums on the
 // warp-level 8-bit integer MMA (mma.sync m16n8k32 s8, codes sign-extended in
-// registers) and applies the two group scales on the FMA pipe.  That combine
-// step -- two packed operations per output element and group -- bounds the
-// kernel; the format is served for correctness and portability of
+// registers) and applies the two group scales on the FMA pipe.  The CUDA-core
+// work around the MMAs -- the sign extension and this two-scale combine --
+// bounds the kernel; the format is served for correctness and portability of
 // checkpoints, NVFP4 is the path the hardware is built for.
 #pragma once
 
