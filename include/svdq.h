@@ -243,7 +243,8 @@ svdq_status svdq_linear_forward(const uint16_t* X, int M, const svdq_weight* w, 
  * back to the host runs on a second, library-owned stream (one per device,
  * created on first use) while the next chunk is copied in and computed, and
  * `stream` then waits for the last copy.  ws is sized for M as for
- * svdq_linear_forward. */
+ * svdq_linear_forward.  SVDQ_HOST_CHUNK_ROWS (a multiple of 128) overrides the
+ * chunk size. */
 svdq_status svdq_linear_forward_host(const uint16_t* X_host, int M, const svdq_weight* w,
                                      uint16_t* Y_host, uint16_t* X_dev, uint16_t* Y_dev,
                                      void* ws, size_t ws_bytes, void* stream);

@@ -1083,7 +1083,12 @@ svdq_status svdq_linear_forward_host(const uint16_t* X_host, int M, const svdq_w
   if (ws_bytes < act_ws_layout(M, w->K, w->r, nullptr, nullptr)) return SVDQ_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t K = w->K, N = w->N;
-  constexpr int kChunk = 1024;   // token rows per pipelined chunk (a multiple of 128)
+  // token rows per pipelined chunk (a multiple of 128); SVDQ_HOST_CHUNK_ROWS overrides
+  int kChunk = 1024;
+  if (const char* e = std::getenv("SVDQ_HOST_CHUNK_ROWS")) {
+    const int v = std::atoi(e);
+    if (v >= 128 && v % 128 == 0) kChunk = v;
+  }
   if (M <= kChunk) {
     SVDQ_CUDA(cudaMemcpyAsync(X_dev, X_host, static_cast<size_t>(M) * K * 2, cudaMemcpyHostToDevice, st));
     s = svdq_linear_forward(X_dev, M, w, Y_dev, ws, ws_bytes, stream);
