@@ -68,8 +68,10 @@ __host__ __device__ __forceinline__ size_t l1_fragment_word(int k, int j, int r)
   return ((static_cast<size_t>(g) * (r >> 3) + t) * 32 + lane) * 2 + h;
 }
 
+// Two CTAs per SM; at r = 64 one, whose 190 registers hold the 32 D accumulators
+// without spilling (128 registers spilled and took 55 instead of 31 us on qkv).
 template <int R_PAD>
-__global__ void __launch_bounds__(ACT_THREADS, 2)
+__global__ void __launch_bounds__(ACT_THREADS, R_PAD > 32 ? 1 : 2)
     act_quant_kernel(const __grid_constant__ CUtensorMap tm_x, const ActParams p) {
   constexpr int kNT = R_PAD / 8;   // n8 tiles (upper bound; the weight holds r/8)
   extern __shared__ uint8_t smem_raw[];
