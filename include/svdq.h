@@ -281,8 +281,9 @@ svdq_status svdq_linear_forward_noalloc(const uint16_t* X, int M, const svdq_wei
 /* ---------------------------------------------------------------------------
  * Test / checkpoint path: copy a prepared weight to host buffers in logical
  * layouts (codes N x K/2, scales N x K/16 row-major, L1 K x r, L2t N x r,
- * inv_lambda K).  Any host pointer may be NULL to skip that field.
- * Synchronises `stream`.
+ * inv_lambda K).  For an INT4 weight the scales are N x K/64 fp16 (uint16
+ * bit patterns, N * K / 32 bytes), row-major.  Any host pointer may be NULL to
+ * skip that field.  Synchronises `stream`.
  * ------------------------------------------------------------------------- */
 svdq_status svdq_weight_export(const svdq_weight* w, uint8_t* host_codes, uint8_t* host_scales,
                                uint16_t* host_L1, uint16_t* host_L2t, float* host_inv_lambda,
@@ -290,9 +291,10 @@ svdq_status svdq_weight_export(const svdq_weight* w, uint8_t* host_codes, uint8_
 
 /* Checkpoint import, the inverse of svdq_weight_export: fill a bound weight
  * from host buffers in the same logical layouts (codes N x K/2, scales
- * N x K/16 row-major, L1 K x r, L2t N x r, inv_lambda K) plus the bias (N
- * bf16; required exactly when w->has_bias).  The scales are converted to the
- * tile layout on the host and L1t is regenerated from L1 on the device.  The
+ * N x K/16 row-major -- N x K/64 fp16 for an INT4 weight -- L1 K x r, L2t N x r,
+ * inv_lambda K) plus the bias (N bf16; required exactly when w->has_bias).  The
+ * scales are converted to the native layout on the host and L1f is regenerated
+ * from L1 on the device.  The
  * watch-ia.com page's offline loop ("quantise, package, load and verify")
  * needs this load step.  Synchronises `stream`.  SVDQ_ERR_INVALID_ARG for a
  * missing buffer. */
