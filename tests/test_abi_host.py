@@ -188,3 +188,13 @@ def test_act_scales_to_logical_is_the_same_conversion():
     a = np.empty_like(logical)
     svdq.svdq_act_scales_to_logical(native.ctypes.data, rows, K, a.ctypes.data)
     assert np.array_equal(a, logical)
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """No CPU fallback: without the shared library every call raises."""
+    monkeypatch.setattr(binding, "LIB_PATH", str(tmp_path / "absent.so"))
+    monkeypatch.setattr(binding, "_lib", None)
+    with pytest.raises(RuntimeError, match="is missing"):
+        binding.svdq_weight_bytes(256, 512, 32, 1)
+    with pytest.raises(RuntimeError, match="is missing"):
+        binding.svdq_version()
