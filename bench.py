@@ -532,11 +532,17 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return None
-    from oracle import svdq_ref as ref
+    from oracle import int4_ref
+    from oracle import svdq_ref
     from workloads import gen
     spec = gen.workload(args.workload)
     d = gen.make_linear(spec)
-    prep = ref.prepare_weight(d["W"], d["lam"], d["bias"], spec.r)   # offline, untimed
+    if args.format == "int4":
+        ref = _Int4OracleView(int4_ref)
+        prep = int4_ref.prepare_weight_int4(d["W"], d["lam"], d["bias"], spec.r)   # offline, untimed
+    else:
+        ref = svdq_ref
+        prep = svdq_ref.prepare_weight(d["W"], d["lam"], d["bias"], spec.r)        # offline, untimed
     rows = args.ref_rows
     X = d["X"][:rows]
     for _ in range(args.warmup):
@@ -556,7 +562,7 @@ def run_reference(args):
         "data": "synthetic (seeded DiT-shaped inputs; no checkpoint)",
         "config": {"workload": f"{spec.name}: DiT joint-attention QKV projection at 1024x1024"
                                if spec.name == "qkv" else spec.name,
-                   "M": spec.M, "K": spec.K, "N": spec.N, "r": spec.r,
+                   "M": spec.M, "K": spec.K, "N": spec.N, "r": spec.r, "format": args.format,
                    "parallelism": "host cores (CPU oracle)"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
                          "sample": f"{rows} of {spec.M} token rows per step, full K and N"},

@@ -45,9 +45,10 @@ def test_cpu_baseline_leg(fmt):
     assert "8 of 256 token rows" in out["sample"]
 
 
-def test_reference_arm_json_line(capsys):
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4"])
+def test_reference_arm_json_line(capsys, fmt):
     out = bench.main(["--impl", "reference", "--workload", "small", "--steps", "1", "--warmup", "3",
-                      "--ref-rows", "8"])
+                      "--ref-rows", "8", "--format", fmt])
     line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
     assert line == json.loads(json.dumps(out))
     for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
@@ -57,7 +58,7 @@ def test_reference_arm_json_line(capsys):
     assert line["impl"] == "reference" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
     assert line["cpu_baseline"]["value"] == line["value"]
-    assert line["config"]["workload"].startswith("small")
+    assert line["config"]["workload"].startswith("small") and line["config"]["format"] == fmt
 
 
 def test_warmup_below_three_is_refused():
