@@ -43,6 +43,7 @@ sys.path.insert(0, ROOT)
 METRIC = "SVDQ W4A4 linear TFLOP/s and % of B200 FP4 tensor peak (HBM % at small M)"
 UNIT = "TFLOP/s"
 FP4_SPEC_TFLOPS = 9000.0          # dense NVFP4, NVIDIA B200 datasheet
+HBM_SPEC_GBS = 8000.0             # HBM3e, NVIDIA B200 datasheet (DGX figure)
 FP4_OVER_BF16 = 4.0               # nominal dense ratio fp4 : bf16 (9 / 2.25 PFLOP/s)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 _CSRC = os.path.join(ROOT, "w4a4_rank_corrected_act_b200", "csrc")
@@ -183,6 +184,64 @@ def _run_for(seconds, flush, step):
             step()
         torch.cuda.synchronize()
 
+def kernel_rooflines(M, N, K, r, gemm_ms, act_ms, int4, workload):
+    """Roofline entries of the GEMM (the dominant kernel) and the activation
+    kernel from their event-timed launch durations (ms): algorithmic bytes or
+    flops per launch over the duration, against the measured peaks."""
+    flops = 2.0 * M * N * K
+    peaks, peak_kind = _peaks()
+    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+    gemm_tflops = flops / (gemm_ms * 1e-3) / 1e12
+    # scale bytes per element: one E4M3 per 16 (NVFP4) or one fp16 per 64 (INT4)
+    sc_div = 32 if int4 else 16
+    act_bytes = M * K * 2 + K * 4 + K * r * 2 + M * K // 2 + M * K // sc_div + M * r * 2
+    act_gbs = act_bytes / (act_ms * 1e-3) / 1e9
+    # the GEMM's own algorithmic bytes: activation codes, scales and D in; the
+    # weight's codes, scales, L2^T and bias in; Y out
+    gemm_bytes = (M * K // 2 + M * K // sc_div + M * r * 2 + N * K // 2 + N * K // sc_div + N * r * 2
+                  + N * 2 + M * N * 2)
+    ridge = fp4_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)        # flop per byte
+    if int4:
+        i8_peak = peaks["bf16_tflops"] * I8_OVER_BF16
+        roofline = {
+            "kernel": "int4_gemm_kernel", "bound": "tensor", "achieved": round(gemm_tflops, 1),
+            "peak": round(i8_peak, 1), "unit": "TFLOP/s", "frac": round(gemm_tflops / i8_peak, 4),
+            "peak_source": f"{peak_kind} bf16 burst {peaks['bf16_tflops']} x nominal int8:bf16 ratio 2",
+            "algorithmic_flops_per_launch": flops,
+        }
+    elif flops / gemm_bytes >= ridge:
+        roofline = {
+            "kernel": "fp4_gemm_kernel", "bound": "tensor", "achieved": round(gemm_tflops, 1),
+            "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(gemm_tflops / fp4_peak, 4),
+            "peak_source": f"{peak_kind} bf16 burst {peaks['bf16_tflops']} x nominal fp4:bf16 ratio 4",
+            "frac_of_fp4_spec_9pf": round(gemm_tflops / FP4_SPEC_TFLOPS, 4),
+            "algorithmic_flops_per_launch": flops,
+        }
+    else:   # below the ridge (small M): weight streaming, against HBM
+        gemm_gbs = gemm_bytes / (gemm_ms * 1e-3) / 1e9
+        roofline = {
+            "kernel": "fp4_gemm_kernel", "bound": "hbm", "achieved": round(gemm_gbs, 1),
+            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(gemm_gbs / peaks["hbm_gbs"], 4),
+            "peak_source": f"{peak_kind} HBM copy",
+            "frac_of_hbm_spec_8000": round(gemm_gbs / HBM_SPEC_GBS, 4),
+            "tflops": round(gemm_tflops, 2),
+        }
+    roofline.update({
+        "traffic": (_profile_traffic(INT4_SRC, f"int4_gemm_{workload}.txt") if int4 else
+                    _profile_traffic(GEMM_SRC, f"fp4_gemm_{workload}.txt")),
+        "algorithmic_bytes_per_launch": gemm_bytes,
+        "arithmetic_intensity_flop_per_byte": round(flops / gemm_bytes, 1),
+        "launch_us": round(gemm_ms * 1e3, 2),
+    })
+    act = {"kernel": "act_quant_int4_kernel" if int4 else "act_quant_kernel", "bound": "hbm",
+           "achieved": round(act_gbs, 1),
+           "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(act_gbs / peaks["hbm_gbs"], 4),
+           "algorithmic_bytes_per_launch": act_bytes, "launch_us": round(act_ms * 1e3, 2),
+           "traffic": (_profile_traffic(INT4_SRC, f"act_quant_int4_{workload}.txt") if int4 else
+                       _profile_traffic(ACT_SRC, f"act_quant_{workload}.txt"))}
+    return roofline, act, fp4_peak
+
+
 def run_native(args):
     import torch
     import torch.distributed as dist
@@ -277,55 +336,7 @@ def run_native(args):
     torch.cuda.synchronize()
     act_ms = statistics.mean(s.elapsed_time(e) for s, e in ev[:reps])
     gemm_ms = statistics.mean(s.elapsed_time(e) for s, e in ev[reps:])
-    peaks, peak_kind = _peaks()
-    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
-    gemm_tflops = flops / (gemm_ms * 1e-3) / 1e12
-    # scale bytes per element: one E4M3 per 16 (NVFP4) or one fp16 per 64 (INT4)
-    sc_div = 32 if int4 else 16
-    act_bytes = M * K * 2 + K * 4 + K * r * 2 + M * K // 2 + M * K // sc_div + M * r * 2
-    act_gbs = act_bytes / (act_ms * 1e-3) / 1e9
-    # the GEMM's own algorithmic bytes: activation codes, scales and D in; the
-    # weight's codes, scales, L2^T and bias in; Y out
-    gemm_bytes = (M * K // 2 + M * K // sc_div + M * r * 2 + N * K // 2 + N * K // sc_div + N * r * 2
-                  + N * 2 + M * N * 2)
-    ridge = fp4_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)        # flop per byte
-    if int4:
-        i8_peak = peaks["bf16_tflops"] * I8_OVER_BF16
-        roofline = {
-            "kernel": "int4_gemm_kernel", "bound": "tensor", "achieved": round(gemm_tflops, 1),
-            "peak": round(i8_peak, 1), "unit": "TFLOP/s", "frac": round(gemm_tflops / i8_peak, 4),
-            "peak_source": f"{peak_kind} bf16 burst {peaks['bf16_tflops']} x nominal int8:bf16 ratio 2",
-            "algorithmic_flops_per_launch": flops,
-        }
-    elif flops / gemm_bytes >= ridge:
-        roofline = {
-            "kernel": "fp4_gemm_kernel", "bound": "tensor", "achieved": round(gemm_tflops, 1),
-            "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(gemm_tflops / fp4_peak, 4),
-            "peak_source": f"{peak_kind} bf16 burst {peaks['bf16_tflops']} x nominal fp4:bf16 ratio 4",
-            "frac_of_fp4_spec_9pf": round(gemm_tflops / FP4_SPEC_TFLOPS, 4),
-            "algorithmic_flops_per_launch": flops,
-        }
-    else:   # below the ridge (small M): weight streaming, against HBM
-        gemm_gbs = gemm_bytes / (gemm_ms * 1e-3) / 1e9
-        roofline = {
-            "kernel": "fp4_gemm_kernel", "bound": "hbm", "achieved": round(gemm_gbs, 1),
-            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(gemm_gbs / peaks["hbm_gbs"], 4),
-            "peak_source": f"{peak_kind} HBM copy",
-            "tflops": round(gemm_tflops, 2),
-        }
-    roofline.update({
-        "traffic": (_profile_traffic(INT4_SRC, f"int4_gemm_{args.workload}.txt") if int4 else
-                    _profile_traffic(GEMM_SRC, f"fp4_gemm_{args.workload}.txt")),
-        "algorithmic_bytes_per_launch": gemm_bytes,
-        "arithmetic_intensity_flop_per_byte": round(flops / gemm_bytes, 1),
-        "launch_us": round(gemm_ms * 1e3, 2),
-    })
-    act = {"kernel": "act_quant_int4_kernel" if int4 else "act_quant_kernel", "bound": "hbm",
-           "achieved": round(act_gbs, 1),
-           "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(act_gbs / peaks["hbm_gbs"], 4),
-           "algorithmic_bytes_per_launch": act_bytes, "launch_us": round(act_ms * 1e3, 2),
-           "traffic": (_profile_traffic(INT4_SRC, f"act_quant_int4_{args.workload}.txt") if int4 else
-                       _profile_traffic(ACT_SRC, f"act_quant_{args.workload}.txt"))}
+    roofline, act, fp4_peak = kernel_rooflines(M, N, K, r, gemm_ms, act_ms, int4, args.workload)
 
     # end to end through the public API with host buffers (pinned), per step:
     # H2D of X, the layer, D2H of Y

@@ -64,3 +64,26 @@ def test_reference_arm_json_line(capsys, fmt):
 def test_warmup_below_three_is_refused():
     with pytest.raises(SystemExit):
         bench.main(["--impl", "reference", "--workload", "small", "--warmup", "2"])
+
+
+def test_kernel_rooflines_for_the_three_regimes():
+    peaks, _ = bench._peaks()
+    # qkv, NVFP4: above the ridge -> tensor-bound against bf16 burst x 4
+    g, a, fp4 = bench.kernel_rooflines(4608, 9216, 3072, 32, 0.0707, 0.0225, False, "qkv")
+    assert g["bound"] == "tensor" and g["unit"] == "TFLOP/s" and g["kernel"] == "fp4_gemm_kernel"
+    assert fp4 == pytest.approx(peaks["bf16_tflops"] * 4)
+    assert g["achieved"] == pytest.approx(2 * 4608 * 9216 * 3072 / 70.7e-6 / 1e12, rel=1e-3)
+    assert g["frac"] == pytest.approx(g["achieved"] / g["peak"], rel=1e-3)
+    assert g["algorithmic_bytes_per_launch"] == 109725696
+    assert a["bound"] == "hbm" and a["algorithmic_bytes_per_launch"] == 36777984
+    # small M, NVFP4: below the ridge -> HBM-bound weight streaming
+    g, a, _ = bench.kernel_rooflines(16, 18432, 3072, 32, 0.01885, 0.0102, False, "small_m")
+    assert g["bound"] == "hbm" and g["unit"] == "GB/s"
+    assert g["frac_of_hbm_spec_8000"] == pytest.approx(g["achieved"] / 8000.0, rel=1e-3)
+    # INT4 variant: against the 8-bit integer tensor peak (bf16 x 2)
+    g, a, _ = bench.kernel_rooflines(4608, 9216, 3072, 32, 0.7394, 0.0353, True, "qkv")
+    assert g["kernel"] == "int4_gemm_kernel" and g["peak"] == pytest.approx(peaks["bf16_tflops"] * 2, rel=1e-3)
+    assert a["kernel"] == "act_quant_int4_kernel" and a["algorithmic_bytes_per_launch"] == 36335616
+    for entry in (g, a):
+        t = entry["traffic"]
+        assert t is None or t > 0
