@@ -9,6 +9,9 @@
  * E4M3 scale per 16 consecutive elements along K).  Activations are quantised
  * to NVFP4 on every call; the bulk of the work runs as a 4-bit x 4-bit
  * block-scaled GEMM on the tensor cores and the low-rank correction in 16 bit.
+ * A weight may instead be bound in the layer's INT4 format (signed 4-bit codes,
+ * one fp16 scale per 64 elements; see svdq_weight), which every entry point
+ * then follows.
  *
  * Sources of the operation (web pages on SVDQuant / Nunchaku):
  *   - W4A4, activation outliers migrated into the weights, the hard part as a

@@ -6,7 +6,8 @@ step of the layer runs in Python: if the shared library is missing or cannot be
 loaded, every call raises -- there is no fallback.
 
 `SvdqLinear` is a small convenience owner of one prepared layer whose device
-memory comes from PyTorch (PyTorch is used for memory and streams only).
+memory comes from PyTorch (PyTorch is used for memory and streams only); its
+``format`` is "nvfp4" (default) or "int4".
 """
 from __future__ import annotations
 
