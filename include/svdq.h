@@ -163,6 +163,13 @@ svdq_status svdq_weight_bind_format(void* buf, size_t bytes, int N, int K, int r
 
 /* ---------------------------------------------------------------------------
  * Offline preparation (smoothing, rank-r split, residual NVFP4 pack).
+ * Defined by: outliers migrated from the activations into the weights, then
+ * absorbed by a 16-bit low-rank branch with the rest quantised to 4 bit
+ * (chaosnode.de "Nunchaku Lite", section "Die Technik: SVDQuant";
+ * aiphreaks.com, section "Technical Breakdown and Performance Metrics"); the
+ * weight split into a low-rank component and a residual (imaginepro.ai,
+ * section "Under the Hood"); quantisation as a separate offline step
+ * (watch-ia.com, the diffuse-compressor flow).
  *   W       device, N x K bf16 (nn.Linear weight)
  *   lambda  device, K float32 smoothing factors (> 0, finite), calibrated by
  *           the caller from activation statistics
@@ -183,6 +190,10 @@ svdq_status svdq_prepare_weight(const uint16_t* W, const float* lambda, const ui
 
 /* ---------------------------------------------------------------------------
  * Activation kernel (one HBM pass over X).
+ * Defined by: the activations quantised to 4 bit on every call once the
+ * outliers have moved into the weights ("A4" of W4A4: aiphreaks.com, section
+ * "Technical Breakdown and Performance Metrics"; watch-ia.com, W4A4), and the
+ * 16-bit low-rank branch's input projection (imaginepro.ai, "Under the Hood").
  *   X        device, M x K bf16
  *   x_codes  device, M x K/2 NVFP4 codes of Xhat = f32(X * inv_lambda)
  *   x_scales device, svdq_act_scales_bytes(M, K) bytes, tile layout; rows
@@ -202,8 +213,11 @@ svdq_status svdq_quantize_act(const uint16_t* X, int M, const svdq_weight* w, ui
  * float32 accumulation in tensor memory.  Inputs as produced by
  * svdq_quantize_act; Y device, M x N bf16.  Single CTAs compute 128 x 256
  * output tiles (N % 256 == 0 and at least one tile per SM) or 128 x 128 tiles
- * (SVDQ_GEMM_BN=128|256 overrides); with SVDQ_GEMM_PAIR=1 and N % 256 == 0,
- * CTA pairs compute 256 x 256 tiles with two-CTA MMAs instead.
+ * (SVDQ_OVERRIDE_GEMM_BN replaces that choice).
+ * Defined by: "most operations happen in 4-bit tensor cores, while the
+ * low-rank correction runs in higher precision" (imaginepro.ai practical
+ * guide, section "Under the Hood: 4-Bit Quantization for Diffusion Models");
+ * the 4-bit operands are NVFP4 on B200 (chaosnode.de, "Hardware-Support").
  * With an INT4 weight: Y = bf16(sum_g sx[m,g] sw[n,g] (sum_{k in group g}
  * qx[m,k] qw[n,k]) + D L2 + bias), the integer group sums exact (8-bit integer
  * warp MMA on the sign-extended codes) and the scaling in float32; 128 x 128
@@ -231,7 +245,11 @@ svdq_status svdq_linear_forward_heads(const uint16_t* X, int M, const svdq_weigh
                                       uint16_t* Y, void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
- * Whole layer: svdq_quantize_act then svdq_gemm on `stream`, with the
+ * Whole layer.  Defined by: the SVDQ layer as a drop-in replacement of a
+ * linear layer, run W4A4 at inference (chaosnode.de "Nunchaku Lite",
+ * sections "Die Technik: SVDQuant" and "Nunchaku Lite vs. Original";
+ * aiphreaks.com, section "Technical Breakdown and Performance Metrics").
+ * svdq_quantize_act then svdq_gemm on `stream`, with the
  * activation codes, scales and D placed in the caller's workspace `ws`
  * (svdq_forward_workspace_bytes(M, N, K, r) bytes, device).
  * ------------------------------------------------------------------------- */
@@ -246,8 +264,8 @@ svdq_status svdq_linear_forward(const uint16_t* X, int M, const svdq_weight* w, 
  * back to the host runs on a second, library-owned stream (one per device,
  * created on first use) while the next chunk is copied in and computed, and
  * `stream` then waits for the last copy.  ws is sized for M as for
- * svdq_linear_forward.  SVDQ_HOST_CHUNK_ROWS (a multiple of 128) overrides the
- * chunk size. */
+ * svdq_linear_forward.  SVDQ_OVERRIDE_HOST_CHUNK_ROWS (a multiple of 128)
+ * replaces the chunk size. */
 svdq_status svdq_linear_forward_host(const uint16_t* X_host, int M, const svdq_weight* w,
                                      uint16_t* Y_host, uint16_t* X_dev, uint16_t* Y_dev,
                                      void* ws, size_t ws_bytes, void* stream);
@@ -282,6 +300,8 @@ svdq_status svdq_linear_forward_noalloc(const uint16_t* X, int M, const svdq_wei
                                         uint16_t* Y, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Defined by: the offline flow's "package" step, a quantised checkpoint that
+ * is later loaded and verified (watch-ia.com, the diffuse-compressor flow).
  * Test / checkpoint path: copy a prepared weight to host buffers in logical
  * layouts (codes N x K/2, scales N x K/16 row-major, L1 K x r, L2t N x r,
  * inv_lambda K).  For an INT4 weight the scales are N x K/64 fp16 (uint16
@@ -340,6 +360,31 @@ svdq_status svdq_int4_scales_to_logical(const uint16_t* native, int rows, int ro
                                         uint16_t* logical);
 svdq_status svdq_int4_scales_to_native(const uint16_t* logical, int rows, int rows_pad, int K,
                                        uint16_t* native);
+
+/* ---------------------------------------------------------------------------
+ * Overrides of automatic launch choices, for tests and tuning sweeps.  The
+ * pages have no counterpart: this is test support.  Process-wide (every
+ * device, every thread); value 0 restores the automatic choice.  Nothing else
+ * (no environment variable) changes these choices.
+ *   SVDQ_OVERRIDE_ACT_KSPLIT       CTAs sharing a 16-row block of the
+ *                                  activation kernel (1-8; used when K is a
+ *                                  multiple of 64 x value)
+ *   SVDQ_OVERRIDE_GEMM_BN          GEMM tile width 128 or 256 (256 only when
+ *                                  N % 256 == 0)
+ *   SVDQ_OVERRIDE_HOST_CHUNK_ROWS  rows per chunk of svdq_linear_forward_host
+ *                                  (a multiple of 128)
+ *   SVDQ_OVERRIDE_SMALL_M          1 = never take the small-M GEMM path,
+ *                                  2 = take it whenever the shape allows
+ * Results are identical under every setting up to float32 summation order
+ * (the tests check each against the oracle).  SVDQ_ERR_INVALID_ARG for an
+ * unknown `which` or a negative value.
+ * ------------------------------------------------------------------------- */
+#define SVDQ_OVERRIDE_ACT_KSPLIT 1
+#define SVDQ_OVERRIDE_GEMM_BN 2
+#define SVDQ_OVERRIDE_HOST_CHUNK_ROWS 3
+#define SVDQ_OVERRIDE_SMALL_M 4
+#define SVDQ_OVERRIDE_COUNT 5
+svdq_status svdq_set_override(int which, int value);
 
 /* Synchronise `stream` and report the device status word of the current
  * device: SVDQ_OK, or SVDQ_ERR_TIMEOUT if a kernel gave up a bounded wait

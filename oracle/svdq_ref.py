@@ -23,12 +23,12 @@ single layer):
     section "Hardware-Support"); rank 32 (watch-ia.com, checkpoint name
     "...nvfp4_r32...").
 
-The concrete formula the layer follows is the one stated with the task:
+The layer follows this formula (the pages describe it in words only):
     Y = Xhat L1 L2 + Q4(Xhat) Q4(R)^T + b,   Xhat = X diag(1/lambda),
     R = diag(lambda) W - (L1 L2)^T           (read with W as K x N, see below),
 NVFP4 = E2M1 codes with one E4M3 scale per 16 consecutive elements along K.
 
-Readings where the pages are silent (each listed in the design doc):
+Readings where the pages are silent (numbered R1-R9, the same numbers the kernels cite):
   R1  W is stored N x K (nn.Linear layout, Y = X W^T).  The residual formula
       is read with W taken K x N there, so What = W diag(lambda) (N x K),
       the SVD is of What^T (K x N), L1 L2 ~= What^T and R = What - (L1 L2)^T

@@ -47,21 +47,17 @@ def bf16_ulp(x: np.ndarray) -> np.ndarray:
     return np.where(a > 0, np.maximum(2.0 ** (e - 7), 2.0 ** -133), 2.0 ** -133)
 
 
-def check_y(y_gpu_bits: np.ndarray, y_oracle64: np.ndarray, what: str = "Y", extra=None):
-    """Output bar: every element within 4e-3 rms(Y_oracle) plus 2 bf16 ulps of
-    itself (the bf16 output rounding), plus `extra` when given.
-
-    `extra` (per element) is the propagated tolerance of an upstream
-    intermediate that the oracle recomputes itself: with D checked to
-    tol_D = 1 ulp + 2^-14 sum|Xhat L1| (check_d), the low-rank term moves Y by at
-    most sum_j tol_D[m, j] |L2[j, n]| (see d_propagated_bound)."""
+def check_y(y_gpu_bits: np.ndarray, y_oracle64: np.ndarray, what: str = "Y"):
+    """Output bar: max|Y_gpu - Y_oracle| <= 4e-3 rms(Y_oracle), and no element
+    off by more than 2 bf16 ulps of itself plus that bound.  Y_oracle is the
+    oracle's whole forward (it recomputes the activation codes, scales and D
+    itself) on the library's exported weight.  Returns max|dY| / rms."""
     yg = ref.bf16_to_f64(y_gpu_bits)
     yo = ref.bf16_to_f64(ref.f64_to_bf16(y_oracle64))
     rms = float(np.sqrt(np.mean(y_oracle64 ** 2)))
     err = np.abs(yg - yo)
-    bound = 4e-3 * rms + 2 * bf16_ulp(yo)
-    if extra is not None:
-        bound = bound + extra
+    tol = 4e-3 * rms
+    bound = tol + 2 * bf16_ulp(yo)
     assert np.all(np.isfinite(yg)), f"{what}: non-finite output"
     over = err > bound
     if np.any(over):
@@ -71,11 +67,14 @@ def check_y(y_gpu_bits: np.ndarray, y_oracle64: np.ndarray, what: str = "Y", ext
         raise AssertionError(f"{what}: {int(over.sum())} elements beyond the bound "
                              f"(rms {rms:.3e}); (m, n, gpu, oracle, err, bound): {rows}")
     worst = float(err.max()) if err.size else 0.0
+    print(f"{what}: max |dY| / rms = {worst / max(rms, 1e-30):.3e} "
+          f"(bar 4e-3; {int((err > 0).sum())} of {err.size} elements differ)")
     return worst / max(rms, 1e-30)
 
 
 def d_propagated_bound(d_oracle_bits: np.ndarray, d_abs: np.ndarray, L2t_bits: np.ndarray):
-    """sum_j tol_D[m, j] |L2[j, n]|: how far Y may move when D is within its bar."""
+    """sum_j tol_D[m, j] |L2[j, n]|: how far Y may move when D is within its bar.
+    A diagnostic printed beside the Y check, never added to the Y bar."""
     o = ref.bf16_to_f64(d_oracle_bits)
     tol = bf16_ulp(o) + 2.0 ** -14 * d_abs
     return tol @ np.abs(ref.bf16_to_f64(L2t_bits)).T

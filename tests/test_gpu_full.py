@@ -63,9 +63,12 @@ def test_full_size_sampled(name):
     prep = dict(inv_lambda=inv, L1=exp["L1"], L2t=exp["L2t"], w_codes=exp["w_codes"],
                 w_scales=exp["w_scales"], bias=d["bias"])
     o = ref.linear_forward(d["X"], prep, rows=rows)
-    # end to end: the oracle recomputes D itself, so its bar carries D's tolerance
+    # end to end (the oracle recomputes the activation codes, scales and D
+    # itself): the strict bar; D's tolerance pushed through L2 is printed only
     extra = d_propagated_bound(o["D"], o["D_abs"], exp["L2t"])
-    rel = check_y(to_np_u16(Y.view(t.int16))[rows], o["Y64"], name, extra=extra)
+    print(f"{name}: D-propagated allowance (diagnostic, not in the bar): median "
+          f"{float(np.median(extra)):.3e}")
+    rel = check_y(to_np_u16(Y.view(t.int16))[rows], o["Y64"], name)
     # the GEMM alone: the oracle's Y on the GPU's own D, without that allowance
     Dg = D.cpu().numpy().view(np.uint16)[rows]
     y_given_d = (o["Y64"] - ref.bf16_to_f64(o["D"]) @ ref.bf16_to_f64(exp["L2t"]).T
@@ -73,3 +76,31 @@ def test_full_size_sampled(name):
     rel_g = check_y(to_np_u16(Y.view(t.int16))[rows], y_given_d, name + " (GPU D)")
     print(f"{name}: max |dY| / rms = {rel:.2e} end to end, {rel_g:.2e} given D")
     assert svdq.svdq_get_device_status(stream()) == 0
+
+
+@pytest.mark.parametrize("name", ["qkv", "mlp_up", "mlp_down"])
+def test_full_size_factors(name):
+    """The rank-r factors at the workloads' own sizes, where the 32nd and 33rd
+    singular values lie inside the bulk of the spectrum: the product L1 L2 of
+    the exported bf16 factors against the oracle's LAPACK SVD (relative
+    Frobenius), L1's column norms against the singular values, and the sign
+    convention."""
+    spec = gen.workload(name)
+    d = gen.make_linear(spec)
+    r = spec.r
+    lin = svdq.SvdqLinear(dev_u16(d["W"]), dev_f32(d["lam"]), dev_u16(d["bias"]), r=r)
+    exp = lin.export()
+    L1o, L2o, sig = ref.svd_split(ref.smooth_weight(d["W"], d["lam"]), r)
+    L1g = ref.bf16_to_f64(exp["L1"])
+    po = ref.bf16_to_f64(L1o) @ ref.bf16_to_f64(L2o)
+    pg = L1g @ ref.bf16_to_f64(exp["L2t"]).T
+    rel = float(np.linalg.norm(pg - po) / np.linalg.norm(po))
+    cn = np.linalg.norm(L1g, axis=0)
+    sv = float(np.max(np.abs(cn / sig[:r] - 1.0)))
+    gap = float(sig[r - 1] / sig[r] - 1.0)
+    print(f"{name}: ||L1L2 - L1oL2o||_F / ||L1oL2o||_F = {rel:.2e}; max |norm/sigma - 1| = {sv:.2e}; "
+          f"sigma_r / sigma_r+1 - 1 = {gap:.2e}")
+    assert rel <= 1e-2, rel
+    assert sv <= 1e-2, sv
+    for j in range(r):
+        assert L1g[np.argmax(np.abs(L1g[:, j])), j] > 0

@@ -1,12 +1,12 @@
 """GPU parity of the CUDA path against the CPU oracle, through the C ABI.
 
-Bars ("Parity"):
+Bars:
   * activation and weight NVFP4 codes and E4M3 scales: bit-exact;
   * inv_lambda: bit-exact;
   * D: 1 bf16 ulp + 2^-14 * sum|Xhat L1| (float32 accumulation bound);
   * Y: every element within 4e-3 rms(Y_oracle) + 2 bf16 ulps of itself; the oracle
-    runs on the library's own exported weight; where the oracle recomputes D
-    itself, D's own tolerance propagated through L2 is added (d_propagated_bound);
+    runs end to end (its own activation codes, scales and D) on the library's
+    own exported weight; nothing else is added to that bar;
   * the rank-r factors: ||L1 L2 - L1o L2o||_F <= 1e-2 ||L1o L2o||_F against the
     oracle's own SVD (bf16 storage of both sides limits this to ~2e-3).
 """
@@ -17,7 +17,7 @@ import w4a4_rank_corrected_act_b200 as svdq
 from oracle import svdq_ref as ref
 from workloads import gen
 
-from gpu_util import (check_d, check_y, d_propagated_bound, dev_f32, dev_u16, dev_u8, empty_u8,
+from gpu_util import (check_d, check_y, dev_f32, dev_u16, dev_u8, empty_u8,
                       stream, to_np_u16, torch)
 
 pytestmark = pytest.mark.gpu
@@ -133,11 +133,11 @@ def test_act_quant_parity(M, K, r):
 
 @pytest.mark.parametrize("ks", [1, 2, 3, 4, 6, 8])
 @pytest.mark.parametrize("r", [32, 64, 0])
-def test_act_quant_parity_k_split(ks, r, monkeypatch):
+def test_act_quant_parity_k_split(ks, r):
     """Clusters of ks CTAs sharing each 16-row block (the small-M path), each
     CTA one of ks equal K ranges, partial D summed in the first CTA."""
-    monkeypatch.setenv("SVDQ_ACT_KS", str(ks))
-    _act_parity_case(40, 3072, r)
+    with svdq.override(svdq.SVDQ_OVERRIDE_ACT_KSPLIT, ks):
+        _act_parity_case(40, 3072, r)
 
 
 def _act_parity_case(M, K, r):
@@ -225,16 +225,18 @@ def test_prepare_parity(N, K, r, with_bias):
 # S2 + S3: GEMM with fused low-rank branch and bias
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("pair", [False, True], ids=["cta", "pair"])
+@pytest.mark.parametrize("BN", [0, 128], ids=["auto", "bn128"])
 @pytest.mark.parametrize("M,K,N,r", [(256, 512, 512, 32), (1, 256, 128, 16), (129, 768, 384, 32),
                                      (300, 1024, 256, 0), (64, 512, 1024, 64), (513, 256, 640, 8),
-                                     (700, 1280, 768, 48)])
-def test_gemm_parity(M, K, N, r, pair, monkeypatch):
+                                     (700, 1280, 768, 48), (1500, 512, 2048, 32)])
+def test_gemm_parity(M, K, N, r, BN):
     """svdq_gemm on oracle-produced activation codes: isolates the tensor-core GEMM
-    (single-CTA 128-row tiles, or 256 x 256 tiles on CTA pairs)."""
-    if pair and N % 256:
-        pytest.skip("the CTA-pair kernel needs N % 256 == 0")
-    monkeypatch.setenv("SVDQ_GEMM_PAIR", "1" if pair else "0")
+    (128 x 256 or 128 x 128 tiles)."""
+    with svdq.override(svdq.SVDQ_OVERRIDE_GEMM_BN, BN):
+        _gemm_parity_case(M, K, N, r)
+
+
+def _gemm_parity_case(M, K, N, r):
     t = torch()
     X, W, B, lam = _inputs(M, K, N, seed=3 * M + K + N + r)
     lin, exp = _prepare(W, lam, B, r)
@@ -253,12 +255,15 @@ def test_gemm_parity(M, K, N, r, pair, monkeypatch):
     check_y(to_np_u16(Y), o["Y64"], "gemm")
 
 
-@pytest.mark.parametrize("BN", ["128", "256"])
-def test_gemm_output_16_byte_aligned(BN, monkeypatch):
+@pytest.mark.parametrize("BN", [128, 256])
+def test_gemm_output_16_byte_aligned(BN):
     """Y only 16-byte aligned (the interface's minimum): the epilogue's rows go
     out as two 16-byte stores; rows past M (ragged tail) are never written."""
-    monkeypatch.setenv("SVDQ_GEMM_PAIR", "0")
-    monkeypatch.setenv("SVDQ_GEMM_BN", BN)
+    with svdq.override(svdq.SVDQ_OVERRIDE_GEMM_BN, BN):
+        _gemm_16_byte_case()
+
+
+def _gemm_16_byte_case():
     t = torch()
     M, K, N, r = 200, 512, 512, 32
     X, W, B, lam = _inputs(M, K, N, seed=77)
@@ -286,14 +291,10 @@ def test_gemm_output_16_byte_aligned(BN, monkeypatch):
 # whole layer
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("pair", [False, True], ids=["cta", "pair"])
 @pytest.mark.parametrize("M,K,N,r,with_bias", [(256, 512, 512, 32, True), (1, 256, 256, 32, True),
                                                (129, 1024, 384, 16, False), (777, 512, 1280, 64, True),
-                                               (40, 768, 128, 0, False)])
-def test_forward_parity(M, K, N, r, with_bias, pair, monkeypatch):
-    if pair and N % 256:
-        pytest.skip("the CTA-pair kernel needs N % 256 == 0")
-    monkeypatch.setenv("SVDQ_GEMM_PAIR", "1" if pair else "0")
+                                               (40, 768, 128, 0, False), (2000, 768, 2304, 32, True)])
+def test_forward_parity(M, K, N, r, with_bias):
     t = torch()
     X, W, B, lam = _inputs(M, K, N, seed=11 * M + K + N + r)
     bias = B if with_bias else None
@@ -302,8 +303,7 @@ def test_forward_parity(M, K, N, r, with_bias, pair, monkeypatch):
     Y = lin.forward(dev_u16(X).view(t.bfloat16))
     t.cuda.synchronize()
     o = ref.linear_forward(X, prep)
-    extra = d_propagated_bound(o["D"], o["D_abs"], exp["L2t"]) if r else None
-    check_y(to_np_u16(Y.view(t.int16)), o["Y64"], "forward", extra=extra)
+    check_y(to_np_u16(Y.view(t.int16)), o["Y64"], "forward")
 
 
 def test_forward_small_workload_end_to_end():
@@ -316,10 +316,14 @@ def test_forward_small_workload_end_to_end():
     prep = _oracle_prep_from_export(d["W"], d["lam"], d["bias"], exp, spec.r)
     Y = to_np_u16(lin.forward(dev_u16(d["X"]).view(t.bfloat16)).view(t.int16))
     o = ref.linear_forward(d["X"], prep)
-    check_y(Y, o["Y64"], "small", extra=d_propagated_bound(o["D"], o["D_abs"], exp["L2t"]))
+    check_y(Y, o["Y64"], "small")
+    # the loose cross-check: the oracle end to end with its own SVD (LAPACK's
+    # factors instead of the library's), within 2e-2 rms
     own = ref.linear_forward(d["X"], ref.prepare_weight(d["W"], d["lam"], d["bias"], spec.r))["Y64"]
     rms = np.sqrt(np.mean(own ** 2))
-    assert np.max(np.abs(ref.bf16_to_f64(Y) - own)) <= 2e-2 * rms * 10  # loose cross-check
+    dev = float(np.max(np.abs(ref.bf16_to_f64(Y) - own)))
+    print(f"small, oracle's own SVD: max |dY| / rms = {dev / rms:.3e} (bar 2e-2)")
+    assert dev <= 2e-2 * rms
 
 
 @pytest.mark.parametrize("M", [200, 2600])

@@ -73,6 +73,7 @@ SIGNATURES = {
     "svdq_act_scales_to_logical": (_I, [_P, _I, _I, _P]),
     "svdq_int4_scales_to_logical": (_I, [_P, _I, _I, _I, _P]),
     "svdq_int4_scales_to_native": (_I, [_P, _I, _I, _I, _P]),
+    "svdq_set_override": (_I, [_I, _I]),
     "svdq_get_device_status": (_I, [_P, ctypes.POINTER(ctypes.c_uint32)]),
     "svdq_clear_device_status": (_I, [_P]),
     "svdq_selftest_wait_timeout": (_I, [ctypes.c_uint64, _P]),
@@ -248,6 +249,31 @@ def svdq_int4_scales_to_logical(native: int, rows: int, rows_pad: int, K: int, l
 
 def svdq_int4_scales_to_native(logical: int, rows: int, rows_pad: int, K: int, native: int) -> None:
     _call("svdq_int4_scales_to_native", logical, rows, rows_pad, K, native)
+
+
+SVDQ_OVERRIDE_ACT_KSPLIT = 1
+SVDQ_OVERRIDE_GEMM_BN = 2
+SVDQ_OVERRIDE_HOST_CHUNK_ROWS = 3
+SVDQ_OVERRIDE_SMALL_M = 4
+
+
+def svdq_set_override(which: int, value: int) -> None:
+    _call("svdq_set_override", which, value)
+
+
+class override:
+    """Context manager: set one launch-choice override, restore automatic (0) on exit."""
+
+    def __init__(self, which: int, value: int):
+        self.which, self.value = which, value
+
+    def __enter__(self):
+        svdq_set_override(self.which, self.value)
+        return self
+
+    def __exit__(self, *exc):
+        svdq_set_override(self.which, 0)
+        return False
 
 
 def svdq_get_device_status(stream: int = 0) -> int:

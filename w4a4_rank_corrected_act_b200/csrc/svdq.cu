@@ -15,17 +15,19 @@
 #include <cusolverDn.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <set>
+#include <utility>
 #include <string>
 #include <vector>
 
 #include "svdq.h"
 #include "act_quant.cuh"
 #include "fp4_gemm.cuh"
-#include "fp4_gemm_pair.cuh"
 #include "int4.cuh"
 #include "prepare.cuh"
 
@@ -85,6 +87,31 @@ svdq_status check_weight(const svdq_weight* w) {
 }
 
 int m_pad_of(int M) { return (M + 127) / 128 * 128; }
+
+// Process-wide overrides of automatic launch choices (svdq_set_override);
+// 0 = automatic.  Only the explicit ABI call changes them.
+std::atomic<int> g_override[SVDQ_OVERRIDE_COUNT];
+
+int override_value(int which) {
+  return (which > 0 && which < SVDQ_OVERRIDE_COUNT) ? g_override[which].load(std::memory_order_relaxed) : 0;
+}
+
+// Dynamic shared memory above 48 KB has to be enabled for each kernel on each
+// device: the attribute applies to the device that is current when it is
+// set.  Done once per (device, kernel).
+svdq_status opt_in_smem(const void* kernel, uint32_t bytes, const char* what) {
+  static std::mutex mu;
+  static std::set<std::pair<int, const void*>> done;
+  int dev = 0;
+  SVDQ_CUDA(cudaGetDevice(&dev));
+  std::lock_guard<std::mutex> lock(mu);
+  if (done.count({dev, kernel})) return SVDQ_OK;
+  const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(bytes));
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  done.insert({dev, kernel});
+  return SVDQ_OK;
+}
 
 // --------------------------------------------------------------------------
 // TMA descriptor encoding through the driver entry point (no libcuda link).
@@ -175,13 +202,11 @@ int num_sms() {
 template <int R_PAD>
 svdq_status launch_act(const CUtensorMap& tx, const ActParams& p, cudaStream_t st) {
   constexpr uint32_t smem = ActSmem<R_PAD>::kBytes;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [&] {
-    attr_err = cudaFuncSetAttribute(act_quant_kernel<R_PAD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    smem);
-  });
-  if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(act)");
+  {
+    const svdq_status so =
+        opt_in_smem(reinterpret_cast<const void*>(act_quant_kernel<R_PAD>), smem, "cudaFuncSetAttribute(act)");
+    if (so != SVDQ_OK) return so;
+  }
   const int grid = p.M_pad / ACT_ROWS * p.ks;
   // programmatic dependent launch (the kernel waits for its predecessor before
   // touching global memory), and a cluster of ks CTAs per row block when ks > 1
@@ -208,11 +233,11 @@ svdq_status launch_act(const CUtensorMap& tx, const ActParams& p, cudaStream_t s
 // K split of the activation kernel: with few row blocks of 16 (small M), a
 // cluster of ks CTAs shares each block so that more SMs stream X.  The largest
 // ks <= 8 with K % (64 ks) == 0, at least one 64-column sub-tile per warp
-// (K / ks >= 512) and at most one CTA per SM.  SVDQ_ACT_KS=ks overrides it
-// when K % (64 ks) == 0.
+// (K / ks >= 512) and at most one CTA per SM.  SVDQ_OVERRIDE_ACT_KSPLIT
+// (svdq_set_override) replaces it when K % (64 ks) == 0.
 int act_k_split(int M, int K) {
-  if (const char* e = std::getenv("SVDQ_ACT_KS")) {
-    const int v = std::atoi(e);
+  {
+    const int v = override_value(SVDQ_OVERRIDE_ACT_KSPLIT);
     if (v >= 1 && v <= ACT_MAX_KS && K % (ACT_SUB * v) == 0) return v;
   }
   const int blocks = (M + ACT_ROWS - 1) / ACT_ROWS;
@@ -227,13 +252,11 @@ svdq_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUte
                         const CUtensorMap& tl2, const CUtensorMap& ty, const GemmParams& p,
                         cudaStream_t st) {
   using Cfg = GemmCfg<BN>;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [&] {
-    attr_err = cudaFuncSetAttribute(fp4_gemm_kernel<BN, R_PAD>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
-  });
-  if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(gemm)");
+  {
+    const svdq_status so = opt_in_smem(reinterpret_cast<const void*>(fp4_gemm_kernel<BN, R_PAD>),
+                                       Cfg::kSmemBytes, "cudaFuncSetAttribute(gemm)");
+    if (so != SVDQ_OK) return so;
+  }
   const int grid = std::min(p.num_tiles, num_sms());
   // programmatic dependent launch: the kernel may start while the preceding
   // kernel of the stream (the activation kernel) finishes; it waits for it
@@ -270,13 +293,11 @@ svdq_status dispatch_gemm_r(int r_pad, const CUtensorMap& ta, const CUtensorMap&
 template <int R_PAD>
 svdq_status launch_act_int4(const CUtensorMap& tx, const Int4ActParams& p, cudaStream_t st) {
   constexpr uint32_t smem = Int4ActSmem<R_PAD>::kBytes;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [&] {
-    attr_err = cudaFuncSetAttribute(act_quant_int4_kernel<R_PAD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    smem);
-  });
-  if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(act int4)");
+  {
+    const svdq_status so = opt_in_smem(reinterpret_cast<const void*>(act_quant_int4_kernel<R_PAD>), smem,
+                                       "cudaFuncSetAttribute(act int4)");
+    if (so != SVDQ_OK) return so;
+  }
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>(p.M_pad / ACT_ROWS));
   cfg.blockDim = dim3(ACT_THREADS);
@@ -321,13 +342,11 @@ svdq_status quantize_act_int4_impl(const uint16_t* X, int M, const svdq_weight* 
 
 template <int R_PAD>
 svdq_status launch_gemm_int4(const CUtensorMap* maps, const Int4GemmParams& p, cudaStream_t st) {
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [&] {
-    attr_err = cudaFuncSetAttribute(int4_gemm_kernel<R_PAD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    I4_SMEM_BYTES);
-  });
-  if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(gemm int4)");
+  {
+    const svdq_status so = opt_in_smem(reinterpret_cast<const void*>(int4_gemm_kernel<R_PAD>), I4_SMEM_BYTES,
+                                       "cudaFuncSetAttribute(gemm int4)");
+    if (so != SVDQ_OK) return so;
+  }
   const dim3 grid(static_cast<unsigned>((p.M + I4_BM - 1) / I4_BM), static_cast<unsigned>(p.N / I4_BN));
   int4_gemm_kernel<R_PAD><<<grid, I4_THREADS, I4_SMEM_BYTES, st>>>(maps[0], maps[1], maps[2], maps[3], p);
   SVDQ_CHECK_LAUNCH("int4_gemm_kernel");
@@ -397,88 +416,17 @@ svdq_status quantize_act_impl(const uint16_t* X, int M, const svdq_weight* w, ui
   }
 }
 
-template <int R_PAD>
-svdq_status launch_gemm_pair(const CUtensorMap* maps, const GemmPairParams& p, int num_pairs,
-                             cudaStream_t st) {
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [&] {
-    attr_err = cudaFuncSetAttribute(fp4_gemm_pair_kernel<R_PAD>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, GemmPairCfg::kSmemBytes);
-  });
-  if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(gemm pair)");
-  fp4_gemm_pair_kernel<R_PAD><<<2 * num_pairs, GP_THREADS, GemmPairCfg::kSmemBytes, st>>>(
-      maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6], p);
-  SVDQ_CHECK_LAUNCH("fp4_gemm_pair_kernel");
-  return SVDQ_OK;
-}
-
-// 256 x 256 tiles on CTA pairs (see fp4_gemm_pair.cuh).
-svdq_status gemm_pair_impl(const uint8_t* x_codes, const uint8_t* x_scales, const uint16_t* D, int M,
-                           const svdq_weight* w, uint16_t* Y, cudaStream_t st) {
-  const int N = w->N, K = w->K, r = w->r, rp = r_pad_of(r);
-  CUtensorMap maps[7] = {};   // a, b, sfa, sfb, d, l2, y
-  svdq_status s = make_tmap(&maps[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, x_codes, K / 2, M, K / 2, 128, 128,
-                            CU_TENSOR_MAP_SWIZZLE_128B);
-  if (s != SVDQ_OK) return s;
-  s = make_tmap(&maps[1], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->w_codes, K / 2, N, K / 2, 128, 128,
-                CU_TENSOR_MAP_SWIZZLE_128B);
-  if (s != SVDQ_OK) return s;
-  // scale tiles of one 128-row block form a row of K * 8 bytes; a 256-wide K
-  // stage is 2 KB of it (256 elements of 8 bytes)
-  s = make_tmap(&maps[2], CU_TENSOR_MAP_DATA_TYPE_UINT64, x_scales, K, m_pad_of(M) / 128,
-                static_cast<uint64_t>(K) * 8, 256, 1, CU_TENSOR_MAP_SWIZZLE_NONE);
-  if (s != SVDQ_OK) return s;
-  s = make_tmap(&maps[3], CU_TENSOR_MAP_DATA_TYPE_UINT64, w->w_scales, K, N / 128,
-                static_cast<uint64_t>(K) * 8, 256, 2, CU_TENSOR_MAP_SWIZZLE_NONE);
-  if (s != SVDQ_OK) return s;
-  if (r > 0) {
-    s = make_tmap(&maps[4], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, D, r, M, static_cast<uint64_t>(r) * 2, rp,
-                  128, lr_swizzle(rp));
-    if (s != SVDQ_OK) return s;
-    s = make_tmap(&maps[5], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->L2t, r, N,
-                  static_cast<uint64_t>(r) * 2, rp, 128, lr_swizzle(rp));
-    if (s != SVDQ_OK) return s;
-  }
-  s = make_tmap(&maps[6], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, N, M, static_cast<uint64_t>(N) * 2, 16, 32,
-                CU_TENSOR_MAP_SWIZZLE_32B);
-  if (s != SVDQ_OK) return s;
-  GemmPairParams p;
-  p.bias = w->has_bias ? w->bias : nullptr;
-  p.M = M;
-  p.N = N;
-  p.K = K;
-  p.r = r;
-  p.m_tiles = (M + GP_BM - 1) / GP_BM;
-  p.n_tiles = N / GP_BN;
-  p.num_tiles = p.m_tiles * p.n_tiles;
-  p.kblocks = K / GEMM_BK;
-  const int num_pairs = std::max(1, std::min(p.num_tiles, num_sms() / 2));
-  switch (rp) {
-    case 0: return launch_gemm_pair<0>(maps, p, num_pairs, st);
-    case 16: return launch_gemm_pair<16>(maps, p, num_pairs, st);
-    case 32: return launch_gemm_pair<32>(maps, p, num_pairs, st);
-    default: return launch_gemm_pair<64>(maps, p, num_pairs, st);
-  }
-}
-
 // head_dim == 0: Y row-major M x N; else Y head-major [N / head_dim][M][head_dim]
 svdq_status gemm_impl(const uint8_t* x_codes, const uint8_t* x_scales, const uint16_t* D, int M,
                       const svdq_weight* w, uint16_t* Y, cudaStream_t st, int head_dim = 0) {
   if (w->format == SVDQ_FORMAT_INT4) return gemm_int4_impl(x_codes, x_scales, D, M, w, Y, st, head_dim);
-  if (head_dim == 0) {
-    // the CTA-pair kernel (256 x 256 tiles) is used on request (SVDQ_GEMM_PAIR=1)
-    bool pair = false;
-    if (const char* e = std::getenv("SVDQ_GEMM_PAIR")) pair = (std::atoi(e) != 0) && (w->N % 256 == 0);
-    if (pair) return gemm_pair_impl(x_codes, x_scales, D, M, w, Y, st);
-  }
   const int N = w->N, K = w->K, r = w->r, rp = r_pad_of(r);
   const int m_tiles = (M + GEMM_BM - 1) / GEMM_BM;
   // 256-wide tiles when N allows it and there are enough of them to fill the GPU
   int BN = (N % 256 == 0) ? 256 : 128;
   if (BN == 256 && m_tiles * (N / 256) < num_sms()) BN = 128;
-  if (const char* e = std::getenv("SVDQ_GEMM_BN")) {   // tile-width override (128 or 256)
-    const int v = std::atoi(e);
+  {   // tile-width override (svdq_set_override)
+    const int v = override_value(SVDQ_OVERRIDE_GEMM_BN);
     if (v == 128 || (v == 256 && N % 256 == 0)) BN = v;
   }
   CUtensorMap ta{}, tb{}, td{}, tl2{}, ty{};
@@ -821,7 +769,13 @@ const char* svdq_status_string(svdq_status s) {
 
 const char* svdq_last_error_detail(void) { return g_last_error.c_str(); }
 
-const char* svdq_version(void) { return "svdq-b200 0.1 (sm_100a)"; }
+const char* svdq_version(void) { return "svdq-b200 0.2 (sm_100a)"; }
+
+svdq_status svdq_set_override(int which, int value) {
+  if (which <= 0 || which >= SVDQ_OVERRIDE_COUNT || value < 0) return SVDQ_ERR_INVALID_ARG;
+  g_override[which].store(value, std::memory_order_relaxed);
+  return SVDQ_OK;
+}
 
 size_t svdq_weight_bytes(int N, int K, int r, int has_bias) {
   if (check_layer_shape(N, K, r) != SVDQ_OK) return 0;
@@ -1083,10 +1037,10 @@ svdq_status svdq_linear_forward_host(const uint16_t* X_host, int M, const svdq_w
   if (ws_bytes < act_ws_layout(M, w->K, w->r, nullptr, nullptr)) return SVDQ_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t K = w->K, N = w->N;
-  // token rows per pipelined chunk (a multiple of 128); SVDQ_HOST_CHUNK_ROWS overrides
+  // token rows per pipelined chunk (a multiple of 128); SVDQ_OVERRIDE_HOST_CHUNK_ROWS replaces it
   int kChunk = 1024;
-  if (const char* e = std::getenv("SVDQ_HOST_CHUNK_ROWS")) {
-    const int v = std::atoi(e);
+  {
+    const int v = override_value(SVDQ_OVERRIDE_HOST_CHUNK_ROWS);
     if (v >= 128 && v % 128 == 0) kChunk = v;
   }
   if (M <= kChunk) {
