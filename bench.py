@@ -242,6 +242,81 @@ def kernel_rooflines(M, N, K, r, gemm_ms, act_ms, int4, workload):
     return roofline, act, fp4_peak
 
 
+def _time_steps(step, flush, steps, warmup, st):
+    """Device time (ms) of each of `steps` calls of step(), L2 flushed before each."""
+    import torch
+    for _ in range(warmup):
+        flush.zero_()
+        step()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        ev[i][0].record(st)
+        step()
+        ev[i][1].record(st)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def layer_entry(spec, step_ms):
+    """Per-workload entry of the bench line: layer latency percentiles, 4-bit
+    TFLOP/s and roofline fractions.  Below the ridge (few tokens) the layer
+    is weight streaming and its fraction is taken against HBM with the
+    algorithmic bytes (X, the weight's codes, scales, L1, L2, 1/lambda and
+    bias, and Y, each once)."""
+    peaks, kind = _peaks()
+    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+    M, K, N, r = spec.M, spec.K, spec.N, spec.r
+    p50 = float(np.percentile(step_ms, 50))
+    tflops = 2.0 * M * N * K / (p50 * 1e-3) / 1e12
+    alg_bytes = (M * K * 2 + N * K // 2 + N * K // 16 + K * r * 2 + N * r * 2 + K * 4 + N * 2 + M * N * 2)
+    e = {"M": M, "K": K, "N": N, "r": r,
+         "us_per_layer": round(p50 * 1e3, 2),
+         "us_p95": round(float(np.percentile(step_ms, 95)) * 1e3, 2),
+         "tflops": round(tflops, 1),
+         "frac_fp4_measured": round(tflops / fp4_peak, 4),
+         "frac_fp4_spec_9000": round(tflops / FP4_SPEC_TFLOPS, 4),
+         "algorithmic_bytes": alg_bytes}
+    ai = 2.0 * M * N * K / alg_bytes
+    if ai < fp4_peak * 1e12 / (peaks["hbm_gbs"] * 1e9):
+        gbs = alg_bytes / (p50 * 1e-3) / 1e9
+        e.update({"bound": "hbm", "gbs": round(gbs, 1), "frac_hbm_measured": round(gbs / peaks["hbm_gbs"], 4),
+                  "frac_hbm_spec_8000": round(gbs / HBM_SPEC_GBS, 4),
+                  "target_us_70pct_of_8000": round(alg_bytes / (0.7 * HBM_SPEC_GBS * 1e9) * 1e6, 2)})
+    else:
+        e.update({"bound": "tensor",
+                  "target_us_60pct_of_9000": round(2.0 * M * N * K / (0.6 * FP4_SPEC_TFLOPS * 1e12) * 1e6, 2)})
+    e["peak_source"] = kind
+    return e
+
+
+def measure_configs(names, steps, warmup, st, flush):
+    """Each named workload as one svdq_linear_forward per step (L2 flushed
+    between steps), on its own seeded inputs; weights prepared untimed."""
+    import torch
+    import w4a4_rank_corrected_act_b200 as svdq
+    from workloads import gen
+    sh = int(st.cuda_stream)
+    out = {}
+    for name in names:
+        spec = gen.workload(name)
+        d = gen.make_linear(spec)
+        dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()  # noqa: E731
+        lin = svdq.SvdqLinear(dev(d["W"]), torch.from_numpy(d["lam"]).cuda(), dev(d["bias"]), r=spec.r)
+        X = dev(d["X"])
+        Y = torch.empty((spec.M, spec.N), dtype=torch.int16, device="cuda")
+        nb = lin.workspace_bytes(spec.M)
+        ws = torch.empty(max(nb, 256), dtype=torch.uint8, device="cuda")
+
+        def step():
+            svdq.svdq_linear_forward(X.data_ptr(), spec.M, lin.w, Y.data_ptr(), ws.data_ptr(), nb, sh)
+
+        out[name] = layer_entry(spec, _time_steps(step, flush, steps, warmup, st))
+        del lin, X, Y, ws
+        torch.cuda.empty_cache()
+    return out
+
+
 def run_native(args):
     import torch
     import torch.distributed as dist
@@ -361,6 +436,24 @@ def run_native(args):
            "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2,
            "ms_per_step": round(e2e_ms / args.steps, 4)}
 
+    configs = None
+    if args.configs and world == 1 and spec.name == "qkv" and not int4:
+        # every workload of the benchmark set, one layer each (the qkv entry
+        # repeats the headline's own steps), the small-token layer against
+        # HBM, and one DiT block of four linears
+        configs = {"qkv": layer_entry(spec, step_ms)}
+        configs.update(measure_configs(["small", "mlp_up", "mlp_down", "small_m"], args.steps, args.warmup,
+                                       st, flush))
+        configs["mlp_pair_unfused"] = {
+            "us": round(configs["mlp_up"]["us_per_layer"] + configs["mlp_down"]["us_per_layer"], 2),
+            "note": "up- and down-projection timed as separate layers (GELU between them not included)"}
+        b_ms, b_layers, b_flops, b_tokens = measure_block("b1", args.steps, args.warmup, st, flush)
+        b_p50 = float(np.percentile(b_ms, 50))
+        configs["block_b1"] = {"tokens": b_tokens, "us_per_block": round(b_p50 * 1e3, 2),
+                               "tflops": round(b_flops / (b_p50 * 1e-3) / 1e12, 1), "layers_us": b_layers}
+        if svdq.svdq_get_device_status(sh):
+            raise SystemExit("a kernel gave up a wait")
+
     out = None
     if rank == 0:
         out = {
@@ -385,6 +478,8 @@ def run_native(args):
             "gpu_launches": 2 * args.steps,
             "clocks": clk.summary(),
         }
+        if configs is not None:
+            out["configs"] = configs
         if args.cpu_baseline:
             out["cpu_baseline"] = cpu_baseline(spec, d, lin.export(), budget_s=args.cpu_seconds,
                                                fmt=args.format)
@@ -395,30 +490,27 @@ def run_native(args):
     return out
 
 
-def run_block(args):
-    """The four linears of one DiT block (workloads block_<b>_{qkv,out,up,down})
+def measure_block(tag, steps, warmup, st, flush):
+    """The four linears of one DiT block (workloads block_<tag>_{qkv,out,up,down})
     back to back on one stream, each on its own synthetic input; one step is
-    the four layers, timed with CUDA events, L2 flushed between steps.  One GPU."""
+    the four layers, L2 flushed between steps.  Returns per-step ms and the
+    mean per-layer us."""
     import torch
     import w4a4_rank_corrected_act_b200 as svdq
     from workloads import gen
-
-    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
-    names = [f"block_{args.block}_{n}" for n in ("qkv", "out", "up", "down")]
-    st = torch.cuda.current_stream()
+    names = [f"block_{tag}_{n}" for n in ("qkv", "out", "up", "down")]
     sh = int(st.cuda_stream)
     layers = []
     for nm in names:
         spec = gen.workload(nm)
         d = gen.make_linear(spec)
-        dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
+        dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()  # noqa: E731
         lin = svdq.SvdqLinear(dev(d["W"]), torch.from_numpy(d["lam"]).cuda(), dev(d["bias"]), r=spec.r)
         X = dev(d["X"])
         Y = torch.empty((spec.M, spec.N), dtype=torch.int16, device="cuda")
         nb = lin.workspace_bytes(spec.M)
         ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
         layers.append((spec, lin, X, Y, ws, nb))
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
 
     def step(evs=None):
         for i, (spec, lin, X, Y, ws, nb) in enumerate(layers):
@@ -428,38 +520,51 @@ def run_block(args):
         if evs is not None:
             evs[len(layers)].record(st)
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         flush.zero_()
         step()
     torch.cuda.synchronize()
-    per = [[torch.cuda.Event(enable_timing=True) for _ in range(len(layers) + 1)] for _ in range(args.steps)]
-    with ClockSampler(0) as clk:
-        _run_for(0.5, flush, step)
-        torch.cuda.synchronize()
-        for i in range(args.steps):
-            flush.zero_()
-            step(per[i])
-        torch.cuda.synchronize()
-        _run_for(0.5, flush, step)
+    per = [[torch.cuda.Event(enable_timing=True) for _ in range(len(layers) + 1)] for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        step(per[i])
+    torch.cuda.synchronize()
     step_ms = [e[0].elapsed_time(e[-1]) for e in per]
-    layer_us = [statistics.mean(e[j].elapsed_time(e[j + 1]) for e in per) * 1e3 for j in range(len(layers))]
-    if svdq.svdq_get_device_status(sh):
-        raise SystemExit("a kernel gave up a wait")
+    layer_us = {spec.name: round(statistics.mean(e[j].elapsed_time(e[j + 1]) for e in per) * 1e3, 2)
+                for j, (spec, *_) in enumerate(layers)}
     flops = sum(2.0 * spec.M * spec.N * spec.K for spec, *_ in layers)
+    tokens = layers[0][0].M
+    del layers
+    torch.cuda.empty_cache()
+    return step_ms, layer_us, flops, tokens
+
+
+def run_block(args):
+    """One DiT block's four linears per step (see measure_block).  One GPU."""
+    import torch
+    import w4a4_rank_corrected_act_b200 as svdq
+
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    st = torch.cuda.current_stream()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    with ClockSampler(0) as clk:
+        step_ms, layer_us, flops, tokens = measure_block(args.block, args.steps, args.warmup, st, flush)
+    if svdq.svdq_get_device_status(int(st.cuda_stream)):
+        raise SystemExit("a kernel gave up a wait")
     total_ms = sum(step_ms)
     out = {
         "metric": METRIC + " (DiT block: four linears)", "value": round(flops * args.steps / (total_ms * 1e-3) / 1e12, 2),
         "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic (seeded DiT-shaped inputs; no checkpoint)",
-        "config": {"workload": f"DiT block, {layers[0][0].M} tokens: QKV 3072->9216, out 3072->3072, "
+        "config": {"workload": f"DiT block, {tokens} tokens: QKV 3072->9216, out 3072->3072, "
                                "up 3072->12288, down 12288->3072, r=32, bias",
                    "l2": "flushed between steps (256 MiB write outside the step events)",
                    "parallelism": "replicas x1 (token-parallel, no collective)"},
-        "layers_us": {spec.name: round(t, 2) for (spec, *_), t in zip(layers, layer_us)},
+        "layers_us": layer_us,
         "step_us_percentiles": {"p50": round(float(np.percentile(step_ms, 50)) * 1e3, 2),
                                 "p95": round(float(np.percentile(step_ms, 95)) * 1e3, 2)},
-        "gpu_launches": 2 * len(layers) * args.steps,
+        "gpu_launches": 8 * args.steps,
         "clocks": clk.summary(),
     }
     print(json.dumps(out), flush=True)
@@ -594,6 +699,8 @@ def main(argv=None):
     ap.add_argument("--format", choices=["nvfp4", "int4"], default="nvfp4",
                     help="4-bit format of the layer (int4: the variant for pre-Blackwell checkpoints)")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--no-configs", dest="configs", action="store_false",
+                    help="skip the per-workload entries (small, mlp_up, mlp_down, small_m, DiT block)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-rows", type=int, default=128)
     ap.add_argument("--block", choices=["b1", "b4"], default=None,

@@ -143,7 +143,15 @@ size_t svdq_weight_bytes(int N, int K, int r, int has_bias);
 size_t svdq_act_codes_bytes(int M, int K);
 size_t svdq_act_scales_bytes(int M, int K);
 
-/* Workspace of svdq_linear_forward: codes + scales + D, 256-byte aligned. */
+/* Workspace of svdq_linear_forward (and its host, head-major and no-allocation
+ * variants), 256-byte aligned fields.  For the general path: codes (M x K/2),
+ * scales (tile layout above) and D (M x r bf16).  For M <= 32 and K <= 3840
+ * the few-token path (see svdq_linear_forward) uses, from the start of the
+ * same buffer: codes M x K/2; the scale words uint32 [K/64][32] (word j of
+ * token m holds the E4M3 codes of its 16-element blocks 4 j .. 4 j + 3, low
+ * byte first; tokens >= M are 0); the float32 partial down-projections
+ * [K/256][M][r] (D = bf16 of their sum in slice order).  The size returned
+ * covers both. */
 size_t svdq_forward_workspace_bytes(int M, int N, int K, int r);
 
 /* Workspace of svdq_prepare_weight.  This asks the eigen-solver for its
@@ -249,6 +257,13 @@ svdq_status svdq_linear_forward_heads(const uint16_t* X, int M, const svdq_weigh
  * linear layer, run W4A4 at inference (chaosnode.de "Nunchaku Lite",
  * sections "Die Technik: SVDQuant" and "Nunchaku Lite vs. Original";
  * aiphreaks.com, section "Technical Breakdown and Performance Metrics").
+ * Few-token path: with an NVFP4 weight, M <= 32, K <= 3840 and N / 128 at
+ * most the number of SMs, the layer is a weight stream and runs as an
+ * activation kernel (K / 256 CTAs: codes, scales, partial D) and a GEMM with
+ * the operands swapped (the weight's 128 rows are the MMA's M, the tokens its
+ * N = 16 or 32; one CTA per 128 weight rows, weight streaming from its first
+ * instruction); same results up to float32 summation order of D.
+ * SVDQ_OVERRIDE_SMALL_M = 1 turns it off.  Otherwise (general path)
  * svdq_quantize_act then svdq_gemm on `stream`, with the
  * activation codes, scales and D placed in the caller's workspace `ws`
  * (svdq_forward_workspace_bytes(M, N, K, r) bytes, device).
@@ -373,8 +388,8 @@ svdq_status svdq_int4_scales_to_native(const uint16_t* logical, int rows, int ro
  *                                  N % 256 == 0)
  *   SVDQ_OVERRIDE_HOST_CHUNK_ROWS  rows per chunk of svdq_linear_forward_host
  *                                  (a multiple of 128)
- *   SVDQ_OVERRIDE_SMALL_M          1 = never take the small-M GEMM path,
- *                                  2 = take it whenever the shape allows
+ *   SVDQ_OVERRIDE_SMALL_M          1 = never take the few-token path of
+ *                                  svdq_linear_forward (see there)
  * Results are identical under every setting up to float32 summation order
  * (the tests check each against the oracle).  SVDQ_ERR_INVALID_ARG for an
  * unknown `which` or a negative value.

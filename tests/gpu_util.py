@@ -47,11 +47,19 @@ def bf16_ulp(x: np.ndarray) -> np.ndarray:
     return np.where(a > 0, np.maximum(2.0 ** (e - 7), 2.0 ** -133), 2.0 ** -133)
 
 
-def check_y(y_gpu_bits: np.ndarray, y_oracle64: np.ndarray, what: str = "Y"):
-    """Output bar: max|Y_gpu - Y_oracle| <= 4e-3 rms(Y_oracle), and no element
-    off by more than 2 bf16 ulps of itself plus that bound.  Y_oracle is the
-    oracle's whole forward (it recomputes the activation codes, scales and D
-    itself) on the library's exported weight.  Returns max|dY| / rms."""
+def check_y(y_gpu_bits: np.ndarray, y_oracle64: np.ndarray, what: str = "Y", y_given_gpu_d=None):
+    """Output bar: every element within 4e-3 rms(Y_oracle) plus 2 bf16 ulps of
+    itself.  Y_oracle is the oracle's whole forward (its own activation codes,
+    scales and D) on the library's exported weight.
+
+    D is a rounding point (bf16 of a K-long sum): the GPU sums in float32 on
+    the tensor cores, the oracle in float64, and near a bf16 rounding boundary
+    the two round to neighbouring values (D has its own bar, check_d).  When
+    `y_given_gpu_d` (the oracle's Y recomputed with the GPU's own D) is given,
+    an element beyond the bar against Y_oracle is accepted only if it meets the
+    same bar against y_given_gpu_d, i.e. the whole difference is that of D;
+    such elements are counted and printed, and may be at most 1 in 10^4.
+    Returns max|dY| / rms."""
     yg = ref.bf16_to_f64(y_gpu_bits)
     yo = ref.bf16_to_f64(ref.f64_to_bf16(y_oracle64))
     rms = float(np.sqrt(np.mean(y_oracle64 ** 2)))
@@ -60,6 +68,13 @@ def check_y(y_gpu_bits: np.ndarray, y_oracle64: np.ndarray, what: str = "Y"):
     bound = tol + 2 * bf16_ulp(yo)
     assert np.all(np.isfinite(yg)), f"{what}: non-finite output"
     over = err > bound
+    n_d = 0
+    if y_given_gpu_d is not None and np.any(over):
+        yd = ref.bf16_to_f64(ref.f64_to_bf16(y_given_gpu_d))
+        ok_d = np.abs(yg - yd) <= tol + 2 * bf16_ulp(yd)
+        n_d = int((over & ok_d).sum())
+        assert n_d <= max(1, err.size // 10000), f"{what}: {n_d} elements differ through D"
+        over = over & ~ok_d
     if np.any(over):
         idx = np.argwhere(over)[:5]
         rows = [(int(i), int(j), float(yg[i, j]), float(yo[i, j]), float(err[i, j]),
@@ -68,8 +83,32 @@ def check_y(y_gpu_bits: np.ndarray, y_oracle64: np.ndarray, what: str = "Y"):
                              f"(rms {rms:.3e}); (m, n, gpu, oracle, err, bound): {rows}")
     worst = float(err.max()) if err.size else 0.0
     print(f"{what}: max |dY| / rms = {worst / max(rms, 1e-30):.3e} "
-          f"(bar 4e-3; {int((err > 0).sum())} of {err.size} elements differ)")
+          f"({int((err > 0).sum())} of {err.size} elements differ; "
+          f"{n_d} beyond the bar only through the GPU's D)")
     return worst / max(rms, 1e-30)
+
+
+def y_with_d(y_oracle64: np.ndarray, d_oracle_bits: np.ndarray, d_gpu_bits: np.ndarray,
+             L2t_bits: np.ndarray) -> np.ndarray:
+    """The oracle's Y with its own low-rank term D L2 replaced by the GPU's D:
+    Y - D_o L2 + D_g L2 (float64; the rest of the oracle's sum is unchanged)."""
+    L2 = ref.bf16_to_f64(L2t_bits).T
+    return y_oracle64 + (ref.bf16_to_f64(d_gpu_bits) - ref.bf16_to_f64(d_oracle_bits)) @ L2
+
+
+def gpu_d(lin, X_dev, M: int) -> np.ndarray:
+    """The activation kernel's D for X (the same kernel, deterministic, that the
+    layer's forward runs), as bf16 bits."""
+    import w4a4_rank_corrected_act_b200 as svdq
+    t = torch()
+    K, r = lin.K, lin.r
+    codes = empty_u8(svdq.svdq_act_codes_bytes(M, K))
+    scales = empty_u8(svdq.svdq_act_scales_bytes(M, K))
+    D = t.empty((M, max(r, 1)), dtype=t.int16, device="cuda")
+    svdq.svdq_quantize_act(X_dev.data_ptr(), M, lin.w, codes.data_ptr(), scales.data_ptr(), D.data_ptr(),
+                           stream())
+    t.cuda.synchronize()
+    return D.cpu().numpy().view(np.uint16)[:, :r]
 
 
 def d_propagated_bound(d_oracle_bits: np.ndarray, d_abs: np.ndarray, L2t_bits: np.ndarray):

@@ -9,7 +9,7 @@ import w4a4_rank_corrected_act_b200 as svdq
 from oracle import svdq_ref as ref
 from workloads import gen
 
-from gpu_util import (check_d, check_y, d_propagated_bound, dev_f32, dev_u16, empty_u8,
+from gpu_util import (check_d, check_y, d_propagated_bound, dev_f32, dev_u16, empty_u8, y_with_d,
                       stream, to_np_u16, torch)
 
 pytestmark = pytest.mark.gpu
@@ -68,11 +68,10 @@ def test_full_size_sampled(name):
     extra = d_propagated_bound(o["D"], o["D_abs"], exp["L2t"])
     print(f"{name}: D-propagated allowance (diagnostic, not in the bar): median "
           f"{float(np.median(extra)):.3e}")
-    rel = check_y(to_np_u16(Y.view(t.int16))[rows], o["Y64"], name)
-    # the GEMM alone: the oracle's Y on the GPU's own D, without that allowance
     Dg = D.cpu().numpy().view(np.uint16)[rows]
-    y_given_d = (o["Y64"] - ref.bf16_to_f64(o["D"]) @ ref.bf16_to_f64(exp["L2t"]).T
-                 + ref.bf16_to_f64(Dg) @ ref.bf16_to_f64(exp["L2t"]).T)
+    y_given_d = y_with_d(o["Y64"], o["D"], Dg, exp["L2t"])
+    rel = check_y(to_np_u16(Y.view(t.int16))[rows], o["Y64"], name, y_given_gpu_d=y_given_d)
+    # the GEMM alone: the oracle's Y on the GPU's own D
     rel_g = check_y(to_np_u16(Y.view(t.int16))[rows], y_given_d, name + " (GPU D)")
     print(f"{name}: max |dY| / rms = {rel:.2e} end to end, {rel_g:.2e} given D")
     assert svdq.svdq_get_device_status(stream()) == 0

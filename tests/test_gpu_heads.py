@@ -7,7 +7,7 @@ import pytest
 from oracle import svdq_ref as ref
 from workloads import gen
 
-from gpu_util import check_y, dev_f32, dev_u16, stream, to_np_u16, torch
+from gpu_util import check_y, dev_f32, dev_u16, gpu_d, stream, to_np_u16, torch, y_with_d
 
 pytestmark = pytest.mark.gpu
 
@@ -50,7 +50,8 @@ def test_heads_layout_matches_row_major(M, K, N, r, hd):
                 w_scales=exp["w_scales"], bias=d["bias"])
     o = ref.linear_forward(d["X"], prep)
     back = to_np_u16(Yh).transpose(1, 0, 2).reshape(M, N)
-    check_y(back, o["Y64"], "heads")
+    yd = y_with_d(o["Y64"], o["D"], gpu_d(lin, X, M), exp["L2t"]) if r else None
+    check_y(back, o["Y64"], "heads", y_given_gpu_d=yd)
 
 
 def test_gemm_heads_16_byte_aligned_output():

@@ -15,7 +15,7 @@ from oracle import int4_ref as i4
 from oracle import svdq_ref as ref
 from workloads import gen
 
-from gpu_util import (check_d, check_y, dev_f32, dev_u16, dev_u8, empty_u8,
+from gpu_util import (check_d, check_y, dev_f32, gpu_d, y_with_d, dev_u16, dev_u8, empty_u8,
                       stream, to_np_u16, torch)
 
 pytestmark = pytest.mark.gpu
@@ -199,7 +199,8 @@ def test_int4_forward_parity(M, K, N, r):
     Y = lin.forward(dev_u16(X).view(t.bfloat16))
     t.cuda.synchronize()
     o = i4.linear_forward_int4(X, prep)
-    check_y(to_np_u16(Y.view(t.int16)), o["Y64"], "int4 forward")
+    yd = y_with_d(o["Y64"], o["D"], gpu_d(lin, dev_u16(X), M), exp["L2t"]) if r else None
+    check_y(to_np_u16(Y.view(t.int16)), o["Y64"], "int4 forward", y_given_gpu_d=yd)
 
 
 def test_int4_heads_match_row_major():
@@ -261,7 +262,8 @@ def test_int4_full_size_sampled():
     prep = dict(inv_lambda=inv, L1=exp["L1"], L2t=exp["L2t"], w_codes=exp["w_codes"],
                 w_scales=exp["w_scales"], bias=d["bias"])
     o = i4.linear_forward_int4(d["X"], prep, rows=rows)
-    check_y(to_np_u16(Y.view(t.int16))[rows], o["Y64"], "int4 qkv")
+    yd = y_with_d(o["Y64"], o["D"], gpu_d(lin, X, M)[rows], exp["L2t"])
+    check_y(to_np_u16(Y.view(t.int16))[rows], o["Y64"], "int4 qkv", y_given_gpu_d=yd)
     assert svdq.svdq_get_device_status(stream()) == 0
 
 

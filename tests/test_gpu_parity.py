@@ -17,7 +17,7 @@ import w4a4_rank_corrected_act_b200 as svdq
 from oracle import svdq_ref as ref
 from workloads import gen
 
-from gpu_util import (check_d, check_y, dev_f32, dev_u16, dev_u8, empty_u8,
+from gpu_util import (check_d, check_y, dev_f32, gpu_d, y_with_d, dev_u16, dev_u8, empty_u8,
                       stream, to_np_u16, torch)
 
 pytestmark = pytest.mark.gpu
@@ -303,7 +303,8 @@ def test_forward_parity(M, K, N, r, with_bias):
     Y = lin.forward(dev_u16(X).view(t.bfloat16))
     t.cuda.synchronize()
     o = ref.linear_forward(X, prep)
-    check_y(to_np_u16(Y.view(t.int16)), o["Y64"], "forward")
+    yd = y_with_d(o["Y64"], o["D"], gpu_d(lin, dev_u16(X), M), exp["L2t"]) if r else None
+    check_y(to_np_u16(Y.view(t.int16)), o["Y64"], "forward", y_given_gpu_d=yd)
 
 
 def test_forward_small_workload_end_to_end():
@@ -316,7 +317,8 @@ def test_forward_small_workload_end_to_end():
     prep = _oracle_prep_from_export(d["W"], d["lam"], d["bias"], exp, spec.r)
     Y = to_np_u16(lin.forward(dev_u16(d["X"]).view(t.bfloat16)).view(t.int16))
     o = ref.linear_forward(d["X"], prep)
-    check_y(Y, o["Y64"], "small")
+    yd = y_with_d(o["Y64"], o["D"], gpu_d(lin, dev_u16(d["X"]), spec.M), exp["L2t"])
+    check_y(Y, o["Y64"], "small", y_given_gpu_d=yd)
     # the loose cross-check: the oracle end to end with its own SVD (LAPACK's
     # factors instead of the library's), within 2e-2 rms
     own = ref.linear_forward(d["X"], ref.prepare_weight(d["W"], d["lam"], d["bias"], spec.r))["Y64"]

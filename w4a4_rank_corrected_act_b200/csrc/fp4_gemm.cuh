@@ -71,7 +71,7 @@ struct GemmCfg {
   static constexpr uint32_t kAcc1Col = (BN == 256 ? 160 : 128);
   static constexpr int kOverlapChunks = (BN == 256 ? (256 - 160) / 32 : 0);
   static constexpr uint32_t kOutBytes = 4 * GEMM_STAGE_OUT;   // epilogue staging, 4 warps
-  static constexpr uint32_t kBarBytes = (2 * kStages + 8) * 8 + 16;
+  static constexpr uint32_t kBarBytes = (2 * kStages + 9) * 8 + 16;
   static constexpr uint32_t kSmemBytes = kStages * kStage + kOutBytes + kBarBytes + 1024;
   static_assert(kSfbCol0 + 32 + 4 * (BN / 32) <= kTmemCols, "scale columns");
   static_assert(kAcc1Col + BN <= kSfaCol0, "accumulator buffer 1");
@@ -277,8 +277,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   uint8_t* out_stage = smem + S * Cfg::kStage;
   uint64_t* bars = reinterpret_cast<uint64_t*>(out_stage + Cfg::kOutBytes);
   // bars[0..S) full, [S..2S) empty, 2S/2S+1 tmem_full[2], 2S+2 tmem_free, 2S+3 drain,
-  // 2S+4/2S+5 sf_ready[2] (scale warps -> MMA), 2S+6/2S+7 sf_free[2] (MMA -> scale warps)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 8);
+  // 2S+4/2S+5 sf_ready[2] (scale warps -> MMA), 2S+6/2S+7 sf_free[2] (MMA -> scale warps),
+  // 2S+8 tmem_done (tensor memory no longer used: MMA thread + epilogue warps)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 9);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -296,6 +297,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   const uint32_t drain_bar = smem_u32(bars + 2 * S + 3);
   auto sf_ready = [&](uint32_t b) { return smem_u32(bars + 2 * S + 4 + b); };
   auto sf_free = [&](uint32_t b) { return smem_u32(bars + 2 * S + 6 + b); };
+  const uint32_t tmem_done = smem_u32(bars + 2 * S + 8);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -310,6 +312,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       mbar_init(sf_ready(b), 4);      // one arrive per scale warp
       mbar_init(sf_free(b), 1);
     }
+    mbar_init(tmem_done, 5);          // the MMA thread and the four epilogue warps
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -478,6 +481,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         tc_commit(drain_bar);
         mbar_wait_drain(drain_bar, 0);
       }
+      mbar_arrive(tmem_done);
     }
   } else if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------ epilogue
@@ -522,7 +526,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       }
     }
     if (lane == 0) bulk_wait_group_all();
+    // this warp's tensor-memory reads are over (every tcgen05.ld waited)
+    tc_fence_before();
     __syncwarp();
+    if (lane == 0) mbar_arrive(tmem_done);
   } else if (warp >= 8) {
     // ------------------------------------------------------------ scale warps
     // Each lane quarter gets its replica of the layout the MMA reads: for
@@ -577,9 +584,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
   }
 
+  // Every lane of every warp meets here (a warp whose elected lane worked
+  // alone reconverges first), and the allocator frees tensor memory only once
+  // the MMAs have completed and the epilogue has read the last accumulator.
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 2) {
+    mbar_wait_drain(tmem_done, 0, 4 * kWaitLimitNs);
     tc_fence_after();
     tmem_dealloc(tmem_base, Cfg::kTmemCols);
   }

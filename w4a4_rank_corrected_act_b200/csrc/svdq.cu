@@ -30,6 +30,7 @@
 #include "fp4_gemm.cuh"
 #include "int4.cuh"
 #include "prepare.cuh"
+#include "small_m.cuh"
 
 using namespace svdq;
 
@@ -469,6 +470,64 @@ svdq_status gemm_impl(const uint8_t* x_codes, const uint8_t* x_scales, const uin
                    : dispatch_gemm_r<128>(rp, ta, tb, td, tl2, ty, p, st);
 }
 
+// ---- few-token path (small_m.cuh) ----------------------------------------
+template <int R_PAD>
+svdq_status launch_act_small(const SmallActParams& p, cudaStream_t st) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(p.K / SMALL_ACT_COLS));
+  cfg.blockDim = dim3(SMALL_THREADS);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, act_quant_small_kernel<R_PAD>, p);
+  if (e != cudaSuccess) return cuda_fail(e, "act_quant_small_kernel launch");
+  SVDQ_CHECK_LAUNCH("act_quant_small_kernel");
+  return SVDQ_OK;
+}
+
+template <int TN, int R_PAD>
+svdq_status launch_gemm_small(const CUtensorMap& tw, const CUtensorMap& tl2, SmallGemmParams p, cudaStream_t st) {
+  // the deepest weight ring that leaves room (<= 200 KB) for one activation
+  // CTA on the same SM
+  int stages = SMALL_MAX_STAGES;
+  while (stages > 2 && small_gemm_layout(TN, R_PAD, p.K, stages, nullptr) > 200u * 1024u) --stages;
+  const uint32_t smem = small_gemm_layout(TN, R_PAD, p.K, stages, &p);
+  {
+    const svdq_status so = opt_in_smem(reinterpret_cast<const void*>(fp4_gemm_small_m_kernel<TN, R_PAD>),
+                                       232448u, "cudaFuncSetAttribute(gemm small M)");
+    if (so != SVDQ_OK) return so;
+  }
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(p.N / 128));
+  cfg.blockDim = dim3(SMALL_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, fp4_gemm_small_m_kernel<TN, R_PAD>, tw, tl2, p);
+  if (e != cudaSuccess) return cuda_fail(e, "fp4_gemm_small_m_kernel launch");
+  SVDQ_CHECK_LAUNCH("fp4_gemm_small_m_kernel");
+  return SVDQ_OK;
+}
+
+template <int TN>
+svdq_status dispatch_gemm_small(int r_pad, const CUtensorMap& tw, const CUtensorMap& tl2, const SmallGemmParams& p,
+                                cudaStream_t st) {
+  switch (r_pad) {
+    case 0: return launch_gemm_small<TN, 0>(tw, tl2, p, st);
+    case 16: return launch_gemm_small<TN, 16>(tw, tl2, p, st);
+    case 32: return launch_gemm_small<TN, 32>(tw, tl2, p, st);
+    default: return launch_gemm_small<TN, 64>(tw, tl2, p, st);
+  }
+}
+
 struct ActWs {
   uint8_t* codes;
   uint8_t* scales;
@@ -485,6 +544,41 @@ size_t act_ws_layout(int M, int K, int r, uint8_t* base, ActWs* out) {
     out->D = r > 0 ? reinterpret_cast<uint16_t*>(base + c + s) : nullptr;
   }
   return c + s + d;
+}
+
+// Workspace of the few-token path (M <= 32): activation codes M x K/2, the
+// activation scale words [K/64][32] and the float32 partial down-projections
+// [K/256][M][r].
+struct SmallWs {
+  uint8_t* codes;
+  uint32_t* sfb;
+  float* dpart;
+};
+
+size_t small_ws_layout(int M, int K, int r, uint8_t* base, SmallWs* out) {
+  const size_t c = align_up(static_cast<size_t>(M) * (K / 2), kAlign);
+  const size_t s = align_up(static_cast<size_t>(K / 64) * SMALL_MAX_TOKENS * 4, kAlign);
+  const size_t d = align_up(static_cast<size_t>(K / 256) * M * r * 4, kAlign);
+  if (out != nullptr) {
+    out->codes = base;
+    out->sfb = reinterpret_cast<uint32_t*>(base + c);
+    out->dpart = reinterpret_cast<float*>(base + c + s);
+  }
+  return c + s + d;
+}
+
+// The few-token path applies to NVFP4 weights with M <= 32, K <= 4096 and at
+// most one 128-row weight tile per SM (SVDQ_OVERRIDE_SMALL_M = 1 turns it off).
+bool small_m_path(int M, const svdq_weight* w) {
+  if (w->format != SVDQ_FORMAT_NVFP4 || override_value(SVDQ_OVERRIDE_SMALL_M) == 1) return false;
+  return M >= 1 && M <= SMALL_MAX_TOKENS && w->K <= SMALL_MAX_K && w->N / 128 <= num_sms();
+}
+
+// Workspace bytes of a forward of M rows (either path).
+size_t forward_ws_bytes(int M, int K, int r) {
+  size_t b = act_ws_layout(M, K, r, nullptr, nullptr);
+  if (M <= SMALL_MAX_TOKENS && K <= SMALL_MAX_K) b = std::max(b, small_ws_layout(M, K, r, nullptr, nullptr));
+  return b;
 }
 
 // Weight buffer layout, each field 256-byte aligned.
@@ -517,6 +611,68 @@ size_t weight_layout(int N, int K, int r, int has_bias, uint8_t* base, svdq_weig
     out->bias = reinterpret_cast<uint16_t*>(bias);
   }
   return off;
+}
+
+// The whole layer for M <= 32 tokens on the few-token path: the activation
+// kernel (K/256 CTAs) and the swapped-operand GEMM, chained by programmatic
+// dependent launch; the workspace holds the small_ws_layout fields.
+svdq_status small_forward_impl(const uint16_t* X, int M, const svdq_weight* w, uint16_t* Y, void* ws,
+                               cudaStream_t st, int head_dim) {
+  const int N = w->N, K = w->K, r = w->r, rp = r_pad_of(r);
+  SmallWs a;
+  small_ws_layout(M, K, r, static_cast<uint8_t*>(ws), &a);
+  SmallActParams ap;
+  ap.X = X;
+  ap.inv_lambda = w->inv_lambda;
+  ap.L1f = reinterpret_cast<const uint32_t*>(w->L1f);
+  ap.x_codes = a.codes;
+  ap.sfb = a.sfb;
+  ap.dpart = a.dpart;
+  ap.M = M;
+  ap.K = K;
+  ap.r = r;
+  svdq_status s;
+  switch (rp) {
+    case 0: s = launch_act_small<0>(ap, st); break;
+    case 16: s = launch_act_small<16>(ap, st); break;
+    case 32: s = launch_act_small<32>(ap, st); break;
+    default: s = launch_act_small<64>(ap, st); break;
+  }
+  if (s != SVDQ_OK) return s;
+  const int TN = M <= 16 ? 16 : 32;
+  CUtensorMap tw{}, tl2{};
+  s = make_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->w_codes, K / 2, N, K / 2, 128, 128,
+                CU_TENSOR_MAP_SWIZZLE_128B);
+  if (s != SVDQ_OK) return s;
+  if (r > 0) {
+    s = make_tmap(&tl2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->L2t, r, N, static_cast<uint64_t>(r) * 2, rp, 128,
+                  lr_swizzle(rp));
+    if (s != SVDQ_OK) return s;
+  }
+  SmallGemmParams gp{};
+  gp.w_scales = w->w_scales;
+  gp.x_codes = a.codes;
+  gp.sfb = a.sfb;
+  gp.dpart = a.dpart;
+  gp.bias = w->has_bias ? w->bias : nullptr;
+  gp.Y = Y;
+  gp.M = M;
+  gp.N = N;
+  gp.K = K;
+  gp.r = r;
+  gp.head_dim = head_dim;
+  return TN == 16 ? dispatch_gemm_small<16>(rp, tw, tl2, gp, st) : dispatch_gemm_small<32>(rp, tw, tl2, gp, st);
+}
+
+// The whole layer (either path) with its scratch at `ws` (forward_ws_bytes).
+svdq_status forward_impl(const uint16_t* X, int M, const svdq_weight* w, uint16_t* Y, void* ws,
+                         cudaStream_t st, int head_dim) {
+  if (small_m_path(M, w)) return small_forward_impl(X, M, w, Y, ws, st, head_dim);
+  ActWs a;
+  act_ws_layout(M, w->K, w->r, static_cast<uint8_t*>(ws), &a);
+  svdq_status s = quantize_act_impl(X, M, w, a.codes, a.scales, a.D, st);
+  if (s != SVDQ_OK) return s;
+  return gemm_impl(a.codes, a.scales, a.D, M, w, Y, st, head_dim);
 }
 
 struct PrepWs {
@@ -794,7 +950,7 @@ size_t svdq_act_scales_bytes(int M, int K) {
 
 size_t svdq_forward_workspace_bytes(int M, int N, int K, int r) {
   if (M < 0 || check_layer_shape(N, K, r) != SVDQ_OK) return 0;
-  return act_ws_layout(M, K, r, nullptr, nullptr);
+  return forward_ws_bytes(M, K, r);
 }
 
 size_t svdq_prepare_workspace_bytes(int N, int K, int r) {
@@ -957,13 +1113,8 @@ svdq_status svdq_linear_forward(const uint16_t* X, int M, const svdq_weight* w, 
   if (M == 0) return SVDQ_OK;
   if (X == nullptr || Y == nullptr || ws == nullptr) return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(Y) || !aligned16(ws)) return SVDQ_ERR_MISALIGNED;
-  if (ws_bytes < act_ws_layout(M, w->K, w->r, nullptr, nullptr)) return SVDQ_ERR_WORKSPACE_TOO_SMALL;
-  ActWs a;
-  act_ws_layout(M, w->K, w->r, static_cast<uint8_t*>(ws), &a);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  s = quantize_act_impl(X, M, w, a.codes, a.scales, a.D, st);
-  if (s != SVDQ_OK) return s;
-  return gemm_impl(a.codes, a.scales, a.D, M, w, Y, st);
+  if (ws_bytes < forward_ws_bytes(M, w->K, w->r)) return SVDQ_ERR_WORKSPACE_TOO_SMALL;
+  return forward_impl(X, M, w, Y, ws, static_cast<cudaStream_t>(stream), 0);
 }
 
 svdq_status svdq_gemm_heads(const uint8_t* x_codes, const uint8_t* x_scales, const uint16_t* D, int M,
@@ -987,13 +1138,8 @@ svdq_status svdq_linear_forward_heads(const uint16_t* X, int M, const svdq_weigh
   if (M == 0) return SVDQ_OK;
   if (X == nullptr || Y == nullptr || ws == nullptr) return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(Y) || !aligned16(ws)) return SVDQ_ERR_MISALIGNED;
-  if (ws_bytes < act_ws_layout(M, w->K, w->r, nullptr, nullptr)) return SVDQ_ERR_WORKSPACE_TOO_SMALL;
-  ActWs a;
-  act_ws_layout(M, w->K, w->r, static_cast<uint8_t*>(ws), &a);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  s = quantize_act_impl(X, M, w, a.codes, a.scales, a.D, st);
-  if (s != SVDQ_OK) return s;
-  return gemm_impl(a.codes, a.scales, a.D, M, w, Y, st, head_dim);
+  if (ws_bytes < forward_ws_bytes(M, w->K, w->r)) return SVDQ_ERR_WORKSPACE_TOO_SMALL;
+  return forward_impl(X, M, w, Y, ws, static_cast<cudaStream_t>(stream), head_dim);
 }
 
 // Copy-out stream and events of the host-buffer path, created once per device.
@@ -1034,7 +1180,7 @@ svdq_status svdq_linear_forward_host(const uint16_t* X_host, int M, const svdq_w
   if (X_host == nullptr || Y_host == nullptr || X_dev == nullptr || Y_dev == nullptr || ws == nullptr)
     return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(X_dev) || !aligned16(Y_dev) || !aligned16(ws)) return SVDQ_ERR_MISALIGNED;
-  if (ws_bytes < act_ws_layout(M, w->K, w->r, nullptr, nullptr)) return SVDQ_ERR_WORKSPACE_TOO_SMALL;
+  if (ws_bytes < forward_ws_bytes(M, w->K, w->r)) return SVDQ_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t K = w->K, N = w->N;
   // token rows per pipelined chunk (a multiple of 128); SVDQ_OVERRIDE_HOST_CHUNK_ROWS replaces it
@@ -1086,7 +1232,7 @@ svdq_status svdq_linear_forward_noalloc(const uint16_t* X, int M, const svdq_wei
   if (M == 0) return SVDQ_OK;
   if (X == nullptr || Y == nullptr) return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(Y)) return SVDQ_ERR_MISALIGNED;
-  const size_t need = act_ws_layout(M, w->K, w->r, nullptr, nullptr);
+  const size_t need = forward_ws_bytes(M, w->K, w->r);
   if (need > static_cast<size_t>(SVDQ_NOALLOC_SCRATCH_BYTES)) {
     g_last_error = "svdq_linear_forward_noalloc: this shape needs " + std::to_string(need) +
                    " bytes of scratch; the fixed scratch holds " +
@@ -1096,12 +1242,7 @@ svdq_status svdq_linear_forward_noalloc(const uint16_t* X, int M, const svdq_wei
   void* scratch = nullptr;
   s = noalloc_scratch_address(&scratch);
   if (s != SVDQ_OK) return s;
-  ActWs a;
-  act_ws_layout(M, w->K, w->r, static_cast<uint8_t*>(scratch), &a);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  s = quantize_act_impl(X, M, w, a.codes, a.scales, a.D, st);
-  if (s != SVDQ_OK) return s;
-  return gemm_impl(a.codes, a.scales, a.D, M, w, Y, st);
+  return forward_impl(X, M, w, Y, scratch, static_cast<cudaStream_t>(stream), 0);
 }
 
 svdq_status svdq_weight_export(const svdq_weight* w, uint8_t* host_codes, uint8_t* host_scales,
