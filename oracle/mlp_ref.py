@@ -10,7 +10,12 @@ this module states it.  Only ``tests/`` may import it.
 Readings (the pages give no formula for the pair):
   R19 The hidden activation is H = bf16_RNE(gelu_tanh(Y_up)), with Y_up the
       up-projection's bf16 output and gelu_tanh(y) = y/2 (1 + tanh(sqrt(2/pi)
-      (y + 0.044715 y^3))) evaluated in float64 and rounded once.  The
+      (y + 0.044715 y^3))), its value computed in float64 and rounded once.
+      The value is computed through the identity 1 + tanh u = 2 / (1 +
+      e^{-2u}), i.e. gelu_tanh(y) = y / (1 + e^{-2u}): the same function,
+      without the cancellation of 1 + tanh u, which in float64 loses every
+      significant digit once tanh u is within 1e-16 of -1 (y below about
+      -5.5, where H is still a normal bf16 number down to about y = -10).  The
       down-projection then runs on H exactly as a standalone layer would
       (smoothing by its own lambda, NVFP4 or INT4 quantisation, its own D).
       A fused kernel that evaluates GELU in float32 may differ from H by one
@@ -32,9 +37,11 @@ _C = math.sqrt(2.0 / math.pi)
 
 
 def gelu_tanh_f64(y: np.ndarray) -> np.ndarray:
-    """tanh-approximated GELU in float64."""
+    """tanh-approximated GELU in float64, as y / (1 + exp(-2u)) (R19)."""
     y = np.asarray(y, dtype=np.float64)
-    return 0.5 * y * (1.0 + np.tanh(_C * (y + 0.044715 * y ** 3)))
+    u = _C * (y + 0.044715 * y ** 3)
+    with np.errstate(over="ignore"):
+        return y / (1.0 + np.exp(-2.0 * u))
 
 
 def mlp_hidden(y_up_bits: np.ndarray) -> np.ndarray:

@@ -2,6 +2,7 @@
 exact algebraic identity and against the erf GELU (a library routine), and the
 whole pair against a scalar-loop composition of the brute-force twin."""
 import math
+from decimal import Decimal, getcontext
 
 import numpy as np
 import pytest
@@ -31,14 +32,42 @@ def test_gelu_tanh_close_to_the_erf_gelu():
     assert np.min(mlp_ref.gelu_tanh_f64(x)) == pytest.approx(-0.17, abs=0.01)
 
 
-def test_hidden_is_one_rounding_of_the_f64_gelu():
+def _gelu_decimal(y: float) -> float:
+    """y/2 (1 + tanh u) in 60-digit decimal arithmetic, tanh from its exponential
+    definition: an independent evaluation of the function, exact to far below
+    float64 rounding (no cancellation at 60 digits for |u| < 60)."""
+    getcontext().prec = 60
+    pi = Decimal("3.14159265358979323846264338327950288419716939937510582097494")
+    d = Decimal(y)
+    u = (Decimal(2) / pi).sqrt() * (d + Decimal("0.044715") * d ** 3)
+    e = (2 * u).exp()
+    return float(d / 2 * (1 + (e - 1) / (e + 1)))
+
+
+def _gelu_ref(v: float) -> float:
+    return _gelu_decimal(v) if abs(v) < 40 else (v if v > 0 else -0.0)
+
+
+def test_hidden_is_one_rounding_of_the_gelu():
     rng = np.random.default_rng(1)
     y = gen.to_bf16_bits(rng.standard_normal(2000) * 3)
     h = mlp_ref.mlp_hidden(y)
     for yb, hb in zip(y[:200], h[:200]):
         yv = float(ref.bf16_to_f64(np.array([yb]))[0])
-        gv = 0.5 * yv * (1.0 + math.tanh(math.sqrt(2.0 / math.pi) * (yv + 0.044715 * yv ** 3)))
-        assert float(ref.bf16_to_f64(np.array([hb]))[0]) == brute.bf16_round(gv)
+        assert float(ref.bf16_to_f64(np.array([hb]))[0]) == brute.bf16_round(_gelu_ref(yv))
+
+
+def test_hidden_in_the_negative_tail():
+    """Down to y = -12 the tanh-GELU is a tiny, non-zero number (normal bf16 to
+    about y = -10, subnormal below): the oracle's H is the single rounding of it
+    there too, where 1 + tanh u would cancel in float64."""
+    ys = np.concatenate([np.linspace(-12.0, -4.0, 321), [-5.5, -7.8125, -10.0, -10.25]])
+    yb = gen.to_bf16_bits(ys)
+    h = ref.bf16_to_f64(mlp_ref.mlp_hidden(yb))
+    for yv, hv in zip(ref.bf16_to_f64(yb), h):
+        want = brute.bf16_round(_gelu_ref(float(yv)))
+        assert hv == want, (yv, hv, want)
+    assert np.all(h[ref.bf16_to_f64(yb) > -10.0] < 0.0)
 
 
 def _prep(W, lam, bias, r):
@@ -70,8 +99,7 @@ def test_pair_against_brute_force_composition(r):
     up = brute.forward(X.tolist(), W1.tolist(), lam1.tolist(), b1.tolist(), p1["L1"].tolist(),
                        p1["L2"].tolist())
     y_up = [[brute.bf16_round(v) for v in row] for row in up["Y64"]]
-    h = [[brute.bf16_round(0.5 * v * (1.0 + math.tanh(math.sqrt(2.0 / math.pi) * (v + 0.044715 * v ** 3))))
-          for v in row] for row in y_up]
+    h = [[brute.bf16_round(_gelu_ref(v)) for v in row] for row in y_up]
     assert np.array_equal(ref.bf16_to_f64(out["H"]), np.array(h))
     down = brute.forward(out["H"].tolist(), W2.tolist(), lam2.tolist(), b2.tolist(), p2["L1"].tolist(),
                          p2["L2"].tolist())
