@@ -286,6 +286,40 @@ svdq_status svdq_linear_forward_host(const uint16_t* X_host, int M, const svdq_w
                                      void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * MLP pair: up-projection, GELU, down-projection, both SVDQ layers, with the
+ * GELU and the down-projection's activation quantisation fused into the
+ * up-projection's epilogue.  Defined by: the original engine's model-specific
+ * fused GELU / MLP kernels (chaosnode.de "Nunchaku Lite", section "Nunchaku
+ * Lite vs. Original"); each linear as in svdq_linear_forward.
+ *   H    = bf16(gelu_tanh(Y_up)),  Y_up = the up-projection's bf16 output,
+ *          gelu_tanh(y) = y/2 (1 + tanh(sqrt(2/pi) (y + 0.044715 y^3))),
+ *          evaluated in float32 as y / (1 + exp(-2u)) (the same function);
+ *   Y    = the down-projection of H (its own smoothing, NVFP4 codes and D).
+ * The up-projection's GEMM writes, per 16 hidden columns of a row, the
+ * down-projection's NVFP4 codes and scale of Hhat = f32(H / lambda_down)
+ * straight into that layer's activation buffers, and accumulates its
+ * D = bf16(sum_k bf16(Hhat) L1_down) in float32 (tensor-core partials per
+ * tile, added across tiles); H itself never crosses HBM.
+ *   X      device, M x K bf16 (K = up->K)
+ *   up     NVFP4 weight, N = F (the hidden width);  down: NVFP4, K = F, r <= 32
+ *          (SVDQ_ERR_UNSUPPORTED_SHAPE otherwise; INVALID_ARG if K != F)
+ *   Y      device, M x down->N bf16
+ *   H_out  optional device M x F bf16: H is also written there (NULL: not)
+ *   ws     device, svdq_mlp_workspace_bytes(M, K, F, down->N, up->r, down->r)
+ *          bytes: the up-projection's activation workspace (the general
+ *          layout of svdq_forward_workspace_bytes(M, F, K, up->r) bytes), the
+ *          down-projection's (codes M x F/2, scales, D; the general layout of
+ *          svdq_forward_workspace_bytes(M, N, F, down->r) bytes, both rounded
+ *          up to 256), then M x down->r float32.
+ * Asynchronous on `stream`; the two GEMMs' results equal the unfused pair's
+ * up to the float32 evaluation of GELU (one bf16 step of H next to a rounding
+ * boundary) and the summation order of D.
+ * ------------------------------------------------------------------------- */
+size_t svdq_mlp_workspace_bytes(int M, int K, int F, int N, int r_up, int r_down);
+svdq_status svdq_mlp_forward(const uint16_t* X, int M, const svdq_weight* up, const svdq_weight* down, uint16_t* Y,
+                             uint16_t* H_out, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Whole layer for callers that cannot allocate device memory.  The pages have
  * no counterpart of this entry point: it is an interface convenience.
  *

@@ -64,6 +64,8 @@ SIGNATURES = {
     "svdq_linear_forward_noalloc": (_I, [_P, _I, _WP, _P, _P]),
     "svdq_gemm_heads": (_I, [_P, _P, _P, _I, _WP, _I, _P, _P]),
     "svdq_linear_forward_heads": (_I, [_P, _I, _WP, _I, _P, _P, _SZ, _P]),
+    "svdq_mlp_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I, _I]),
+    "svdq_mlp_forward": (_I, [_P, _I, _WP, _WP, _P, _P, _P, _SZ, _P]),
     "svdq_weight_export": (_I, [_WP, _P, _P, _P, _P, _P, _P]),
     "svdq_weight_import": (_I, [_WP, _P, _P, _P, _P, _P, _P, _P]),
     "svdq_calib_absmax": (_I, [_P, _I, _I, _P, _P]),
@@ -208,6 +210,18 @@ def svdq_linear_forward_noalloc(X: int, M: int, w: svdq_weight, Y: int, stream: 
         raise SvdqError("svdq_linear_forward_noalloc", st,
                         lib().svdq_last_error_detail().decode(errors="replace"))
     _check("svdq_linear_forward_noalloc", st)
+
+
+def svdq_mlp_workspace_bytes(M: int, K: int, F: int, N: int, r_up: int, r_down: int) -> int:
+    return int(lib().svdq_mlp_workspace_bytes(M, K, F, N, r_up, r_down))
+
+
+def svdq_mlp_forward(X: int, M: int, up: svdq_weight, down: svdq_weight, Y: int, H_out: int, ws: int,
+                     ws_bytes: int, stream: int) -> None:
+    """MLP pair (up-projection, GELU, down-projection) with the GELU and the
+    down-projection's activation quantisation in the up-projection's epilogue."""
+    _call("svdq_mlp_forward", X or None, M, ctypes.byref(up), ctypes.byref(down), Y or None, H_out or None,
+          ws or None, ws_bytes, stream or None)
 
 
 def svdq_weight_export(w: svdq_weight, host_codes: int, host_scales: int, host_L1: int,

@@ -44,6 +44,8 @@ struct ActParams {
   uint16_t* D;
   int M, K, r, M_pad;
   int ks;                  // CTAs per cluster sharing a row block (K split); K % (64 ks) == 0
+  float* zero_ptr;         // optional: zero_count floats set to 0 by the grid (the MLP pair's D
+  int zero_count;          // accumulator, which the next kernel of the stream adds into)
 };
 
 template <int R_PAD>
@@ -105,6 +107,8 @@ __global__ void __launch_bounds__(ACT_THREADS, R_PAD > 32 ? 1 : 2)
   // own wait, which waits for this grid to finish.
   pdl_wait();
   pdl_launch_dependents();
+  for (int i = blockIdx.x * ACT_THREADS + threadIdx.x; i < p.zero_count; i += gridDim.x * ACT_THREADS)
+    p.zero_ptr[i] = 0.0f;
   if (row0 >= p.M) {
     // rows entirely in [M, M_pad): their scale entries are written as zero
     // (the whole cluster shares the row block, so every CTA of it leaves here)

@@ -56,7 +56,17 @@ struct GemmParams {
   int head_dim;           // 0: Y row-major; else Y head-major, [N / head_dim][M][head_dim]
   int M, N, K, r;
   int m_tiles, n_tiles, num_tiles, kblocks;
+  // MLP epilogue only (the up-projection of an MLP pair; N is the hidden width F):
+  const float* inv_lambda_next;   // F, 1/lambda of the down-projection
+  const uint32_t* L1f_next;       // the down-projection's L1 (F x r_next) in B-fragment order
+  int r_next;                     // the down-projection's rank, <= 32
+  uint8_t* h_codes;               // M x F/2 NVFP4 codes of the down-projection's smoothed input
+  uint8_t* h_scales;              // their E4M3 scales, tile layout (rows padded to 128, padding 0)
+  float* d_acc;                   // M x r_next float32, zero on entry: sum of bf16(Hhat) L1_next
+  uint16_t* h_out;                // optional M x F bf16: H itself (null: not written)
 };
+
+constexpr int GEMM_MLP_THREADS = 512;   // 4 + 8 epilogue + 4 scale warps
 
 template <int BN>
 struct GemmCfg {
@@ -261,8 +271,168 @@ __device__ __forceinline__ void epilogue_tile(uint32_t acc, uint32_t lane_addr, 
   }
 }
 
-template <int BN, int R_PAD>
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
+// GELU, tanh form, y/2 (1 + tanh u) with u = sqrt(2/pi) (y + 0.044715 y^3),
+// evaluated as y / (1 + e^{-2u}) (the same function: 1 + tanh u = 2 / (1 +
+// e^{-2u})), which keeps its relative accuracy where 1 + tanh u cancels, with
+// the device's exponential and reciprocal.  Where e^{-2u} > e^80 the value is
+// y e^{2u} to float32 precision, taken with the exponential that keeps
+// subnormal results (the value is a subnormal number below about y = -10).
+__device__ __forceinline__ float gelu_tanh_f32(float y) {
+  const float y3 = y * y * y;
+  const float m2u = -1.5957691216057308f * fmaf(0.044715f, y3, y);   // -2u
+  if (m2u > 80.0f) return y * expf(-m2u);
+  float rc;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(rc) : "f"(1.0f + __expf(m2u)));
+  return y * rc;
+}
+
+// MLP epilogue of one 16-column piece of the up-projection's tile for the
+// warp owning rows row0 .. row0 + 31 (lane = row): columns n .. n + 15 of the
+// hidden layer.  For each element: Y_up = bf16(acc + bias); H = bf16(GELU(Y_up));
+// Hhat = f32(H / lambda_next).  The 16 Hhat of the row are one NVFP4 block of
+// the down-projection's input: its 8 code bytes and its scale go straight to
+// that layer's activation buffers.  bf16(Hhat) goes through a per-warp
+// 32 x 16 shared tile into two m16n8k16 A fragments, whose bf16 MMAs with the
+// piece's 16 rows of L1_next accumulate the tile's partial of D_next in dacc.
+template <int NT>
+__device__ __forceinline__ void mlp_piece(const uint32_t (&v)[16], int n, int row, const GemmParams& p,
+                                          uint8_t* dstage, uint32_t dstage_u, int lane, float (&dacc)[2][NT][4],
+                                          uint64_t six, uint64_t neg_y6) {
+  const int F = p.N;
+  // bias and 1/lambda_next of the piece: the same 16 values on every lane
+  float b[16];
+  if (p.bias != nullptr) {
+    const uint4 b0 = __ldg(reinterpret_cast<const uint4*>(p.bias + n));
+    const uint4 b1 = __ldg(reinterpret_cast<const uint4*>(p.bias + n + 8));
+    const uint32_t bw[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      b[2 * i] = bf16_bits_to_f32(bw[i] & 0xFFFFu);
+      b[2 * i + 1] = bf16_bits_to_f32(bw[i] >> 16);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) b[i] = 0.0f;
+  }
+  float inv[16];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float4 x = __ldg(reinterpret_cast<const float4*>(p.inv_lambda_next + n) + i);
+    inv[4 * i] = x.x; inv[4 * i + 1] = x.y; inv[4 * i + 2] = x.z; inv[4 * i + 3] = x.w;
+  }
+  uint32_t hb[8];          // H, packed bf16 pairs
+  uint64_t nh[8];          // -Hhat, packed f32 pairs
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t yb = pack_bf16x2(__uint_as_float(v[2 * i]) + b[2 * i], __uint_as_float(v[2 * i + 1]) + b[2 * i + 1]);
+    const uint32_t h = pack_bf16x2(gelu_tanh_f32(bf16_bits_to_f32(yb & 0xFFFFu)), gelu_tanh_f32(bf16_bits_to_f32(yb >> 16)));
+    hb[i] = h;
+    nh[i] = f32x2_mul(f32x2_pack(bf16_bits_to_f32(h & 0xFFFFu), bf16_bits_to_f32(h >> 16)),
+                      f32x2_pack(-inv[2 * i], -inv[2 * i + 1]));
+  }
+  uint32_t sc;
+  const uint64_t codes = nvfp4_quant_block16_x2(nh, six, neg_y6, sc);
+  if (row < p.M) {
+    *reinterpret_cast<uint64_t*>(p.h_codes + static_cast<size_t>(row) * (F / 2) + n / 2) = codes;
+    if (p.h_out != nullptr) {
+      uint4* dst = reinterpret_cast<uint4*>(p.h_out + static_cast<size_t>(row) * F + n);
+      dst[0] = make_uint4(hb[0], hb[1], hb[2], hb[3]);
+      dst[1] = make_uint4(hb[4], hb[5], hb[6], hb[7]);
+    }
+  }
+  // rows of the last row tile at and beyond M get zero scales (padding)
+  p.h_scales[sf_offset(static_cast<uint32_t>(row), static_cast<uint32_t>(n / 16), static_cast<uint32_t>(F))] =
+      static_cast<uint8_t>(row < p.M ? sc : 0u);
+  // bf16(Hhat) = -bf16(-Hhat) (rounding commutes with negation)
+  uint32_t a8[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float lo, hi;
+    f32x2_unpack(nh[i], lo, hi);
+    a8[i] = pack_bf16x2(lo, hi) ^ 0x80008000u;
+  }
+  __syncwarp();   // the previous piece's fragments have been read
+  *reinterpret_cast<uint4*>(dstage + lane * 32) = make_uint4(a8[0], a8[1], a8[2], a8[3]);
+  *reinterpret_cast<uint4*>(dstage + lane * 32 + 16) = make_uint4(a8[4], a8[5], a8[6], a8[7]);
+  __syncwarp();
+  uint32_t a[2][4];
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+    ldmatrix_x4(dstage_u + (16 * mt + (lane & 15)) * 32 + (lane >> 4) * 16, a[mt][0], a[mt][1], a[mt][2], a[mt][3]);
+  const int nt = p.r_next >> 3;
+  const uint2* f = reinterpret_cast<const uint2*>(p.L1f_next);
+#pragma unroll
+  for (int t = 0; t < NT; ++t) {
+    if (t < nt) {
+      const uint2 bf = __ldg(f + ((static_cast<size_t>(n / 16) * nt + t) * 32 + lane));
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) mma_bf16_16816(dacc[mt][t], a[mt][0], a[mt][1], a[mt][2], a[mt][3], bf.x, bf.y);
+    }
+  }
+}
+
+// MLP epilogue of one 128 x BN tile for one of the two warps of lane quarter
+// q (half h takes the pieces order(h), order(h + 2), ...; the first of them
+// are the columns the next tile's accumulator shares, released after one
+// batched read), then the tile's partial D_next into d_acc.
+template <int BN, int KOV, typename Order, typename Release>
+__device__ __forceinline__ void mlp_epilogue_tile(uint32_t acc, uint32_t lane_addr, int lane, int half, int row0,
+                                                  int n0, const GemmParams& p, uint8_t* dstage, uint32_t dstage_u,
+                                                  Order order, Release release) {
+  constexpr int kMine = BN / 32, kOvMine = KOV / 2, kNT = 4;
+  const int row = row0 + lane;
+  const uint64_t six = f32x2_pack(6.0f, 6.0f);
+  const float y6 = e4m3_table_entry(0x4C).y;   // code 0x4C is 6.0: RN(1/6)
+  const uint64_t neg_y6 = f32x2_pack(-y6, -y6);
+  float dacc[2][kNT][4];
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int t = 0; t < kNT; ++t)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) dacc[mt][t][i] = 0.0f;
+  if constexpr (kOvMine > 0) {
+    uint32_t ov[kOvMine][16];
+#pragma unroll
+    for (int j = 0; j < kOvMine; ++j) tmem_ld_32x32b_x16(acc + lane_addr + order(half + 2 * j) * 16, ov[j]);
+    tmem_ld_wait();
+    tc_fence_before();
+    release();
+#pragma unroll
+    for (int j = 0; j < kOvMine; ++j)
+      mlp_piece<kNT>(ov[j], n0 + 16 * order(half + 2 * j), row, p, dstage, dstage_u, lane, dacc, six, neg_y6);
+  } else {
+    tc_fence_before();
+    release();
+  }
+  for (int j = kOvMine; j < kMine; ++j) {
+    uint32_t v[16];
+    tmem_ld_32x32b_x16(acc + lane_addr + order(half + 2 * j) * 16, v);
+    tmem_ld_wait();
+    mlp_piece<kNT>(v, n0 + 16 * order(half + 2 * j), row, p, dstage, dstage_u, lane, dacc, six, neg_y6);
+  }
+  // the tile's partial D_next: fragment rows lane / 4 (+ 8) of each 16-row
+  // block, columns 8 t + 2 (lane % 4) (+ 1)
+  const int nt = p.r_next >> 3;
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int t = 0; t < kNT; ++t) {
+      if (t >= nt) continue;
+      const int r_lo = row0 + 16 * mt + (lane >> 2), col = 8 * t + 2 * (lane & 3);
+      if (r_lo < p.M) {
+        atomicAdd(p.d_acc + static_cast<size_t>(r_lo) * p.r_next + col, dacc[mt][t][0]);
+        atomicAdd(p.d_acc + static_cast<size_t>(r_lo) * p.r_next + col + 1, dacc[mt][t][1]);
+      }
+      if (r_lo + 8 < p.M) {
+        atomicAdd(p.d_acc + static_cast<size_t>(r_lo + 8) * p.r_next + col, dacc[mt][t][2]);
+        atomicAdd(p.d_acc + static_cast<size_t>(r_lo + 8) * p.r_next + col + 1, dacc[mt][t][3]);
+      }
+    }
+}
+
+template <int BN, int R_PAD, bool MLP = false>
+__global__ void __launch_bounds__(MLP ? GEMM_MLP_THREADS : GEMM_THREADS, 1)
     fp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                     const __grid_constant__ CUtensorMap tm_d, const __grid_constant__ CUtensorMap tm_l2,
                     const __grid_constant__ CUtensorMap tm_y, const GemmParams p) {
@@ -270,6 +440,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   constexpr int S = Cfg::kStages;
   constexpr uint32_t kLRLayout = (R_PAD == 64 ? LAYOUT_SW128 : R_PAD == 32 ? LAYOUT_SW64 : LAYOUT_SW32);
   constexpr uint32_t kLRSbo = 8 * R_PAD * 2;
+  // epilogue warps: 4 (one per lane quarter), or 8 for the MLP epilogue (two
+  // per lane quarter, splitting the tile's columns); the scale warps follow
+  constexpr int kEpiWarps = MLP ? 8 : 4;
+  constexpr int kScaleWarp0 = 4 + kEpiWarps;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -306,13 +480,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
     mbar_init(tmem_full(0), 1);
     mbar_init(tmem_full(1), 1);
-    mbar_init(tmem_free, 4);          // one arrive per epilogue warp
+    mbar_init(tmem_free, kEpiWarps);  // one arrive per epilogue warp
     mbar_init(drain_bar, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(sf_ready(b), 4);      // one arrive per scale warp
       mbar_init(sf_free(b), 1);
     }
-    mbar_init(tmem_done, 5);          // the MMA thread and the four epilogue warps
+    mbar_init(tmem_done, kEpiWarps + 1);   // the MMA thread and the epilogue warps
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -483,7 +657,33 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       }
       mbar_arrive(tmem_done);
     }
-  } else if (warp >= 4 && warp < 8) {
+  } else if (MLP && warp >= 4 && warp < kScaleWarp0) {
+    // --------------------------------------------------------- MLP epilogue
+    const int q = warp & 3, half = (warp - 4) >> 2;
+    uint8_t* dstage = out_stage + (warp - 4) * 1024;
+    const uint32_t dstage_u = smem_u32(dstage);
+    const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+    int local = 0;
+    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++local) {
+      const int mb = t % p.m_tiles, nb = t / p.m_tiles;
+      const int m0 = mb * GEMM_BM, n0 = nb * BN;
+      const int buf = local & 1;
+      const uint32_t acc = tmem_base + (buf ? Cfg::kAcc1Col : 0u);
+      if (!mbar_wait(tmem_full(buf), static_cast<uint32_t>(local >> 1) & 1u, abort_flag, KID_GEMM, 8)) break;
+      tc_fence_after();
+      constexpr int kPieces = BN / 16, kOv = 2 * Cfg::kOverlapChunks;
+      auto order = [&](int i) { return buf ? i : (i + kPieces - kOv) % kPieces; };
+      auto release = [&]() {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tmem_free);
+      };
+      mlp_epilogue_tile<BN, kOv>(acc, lane_addr, lane, half, m0 + q * 32, n0, p, dstage, dstage_u, order, release);
+    }
+    // this warp's tensor-memory reads are over (every tcgen05.ld waited)
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(tmem_done);
+  } else if (!MLP && warp >= 4 && warp < kScaleWarp0) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
     uint8_t* stg = out_stage + q * GEMM_STAGE_OUT;
@@ -530,7 +730,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(tmem_done);
-  } else if (warp >= 8) {
+  } else if (warp >= kScaleWarp0) {
     // ------------------------------------------------------------ scale warps
     // Each lane quarter gets its replica of the layout the MMA reads: for
     // k-block i of a stage, 4 columns of A scales and BN/32 columns of B

@@ -184,6 +184,35 @@ __device__ __forceinline__ uint32_t nvfp4_quant_half_block_x2(const uint64_t (&n
   return e2m1x8_signed(q);
 }
 
+// One whole 16-element block in one thread: the same result as
+// nvfp4_quant_half_block_x2 for the pair of lanes holding its halves, for the
+// 16 values given NEGATED and packed in pairs (nv[u] = (-v[2u], -v[2u+1])).
+// s and RN(1/s) are formed in place (e4m3_table_entry) instead of read from a
+// table.  Returns the 16 codes, element 0 in the lowest nibble.
+__device__ __forceinline__ uint64_t nvfp4_quant_block16_x2(const uint64_t (&nv)[8], uint64_t six, uint64_t neg_y6,
+                                                          uint32_t& scale_code) {
+  float am = 0.0f;
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    float lo, hi;
+    f32x2_unpack(nv[u], lo, hi);
+    am = fmaxf(am, fmaxf(fabsf(lo), fabsf(hi)));
+  }
+  float a6, a6b;
+  f32x2_unpack(quotient_f32x2(f32x2_pack(-am, -am), six, neg_y6), a6, a6b);   // RN(amax / 6)
+  const uint32_t sc = e4m3_rn_satfinite(a6);
+  scale_code = sc;
+  const float2 sy = e4m3_table_entry(sc);
+  const uint64_t s2 = f32x2_pack(sy.x, sy.x), neg_y2 = f32x2_pack(-sy.y, -sy.y);
+  uint64_t q0[4], q1[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    q0[u] = quotient_f32x2(nv[u], s2, neg_y2);
+    q1[u] = quotient_f32x2(nv[u + 4], s2, neg_y2);
+  }
+  return static_cast<uint64_t>(e2m1x8_signed(q0)) | (static_cast<uint64_t>(e2m1x8_signed(q1)) << 32);
+}
+
 // Byte offset of scale (row, kb16) in the scale-factor tile layout:
 // 512-byte tiles of 128 rows x 4 scales, tile (row/128, kb16/4) at
 // ((row/128) * (K/64) + kb16/4) * 512, inside it (row%32)*16 + ((row/32)%4)*4 + kb16%4.

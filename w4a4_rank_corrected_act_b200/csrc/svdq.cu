@@ -248,13 +248,13 @@ int act_k_split(int M, int K) {
   return ks;
 }
 
-template <int BN, int R_PAD>
+template <int BN, int R_PAD, bool MLP = false>
 svdq_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
                         const CUtensorMap& tl2, const CUtensorMap& ty, const GemmParams& p,
                         cudaStream_t st) {
   using Cfg = GemmCfg<BN>;
   {
-    const svdq_status so = opt_in_smem(reinterpret_cast<const void*>(fp4_gemm_kernel<BN, R_PAD>),
+    const svdq_status so = opt_in_smem(reinterpret_cast<const void*>(fp4_gemm_kernel<BN, R_PAD, MLP>),
                                        Cfg::kSmemBytes, "cudaFuncSetAttribute(gemm)");
     if (so != SVDQ_OK) return so;
   }
@@ -264,7 +264,7 @@ svdq_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUte
   // before reading anything that kernel writes
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
-  cfg.blockDim = dim3(GEMM_THREADS);
+  cfg.blockDim = dim3(MLP ? GEMM_MLP_THREADS : GEMM_THREADS);
   cfg.dynamicSmemBytes = Cfg::kSmemBytes;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -272,21 +272,21 @@ svdq_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUte
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, fp4_gemm_kernel<BN, R_PAD>, ta, tb, td, tl2, ty, p);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, fp4_gemm_kernel<BN, R_PAD, MLP>, ta, tb, td, tl2, ty, p);
   if (e != cudaSuccess) return cuda_fail(e, "fp4_gemm_kernel launch");
   SVDQ_CHECK_LAUNCH("fp4_gemm_kernel");
   return SVDQ_OK;
 }
 
-template <int BN>
+template <int BN, bool MLP = false>
 svdq_status dispatch_gemm_r(int r_pad, const CUtensorMap& ta, const CUtensorMap& tb,
                             const CUtensorMap& td, const CUtensorMap& tl2, const CUtensorMap& ty,
                             const GemmParams& p, cudaStream_t st) {
   switch (r_pad) {
-    case 0: return launch_gemm<BN, 0>(ta, tb, td, tl2, ty, p, st);
-    case 16: return launch_gemm<BN, 16>(ta, tb, td, tl2, ty, p, st);
-    case 32: return launch_gemm<BN, 32>(ta, tb, td, tl2, ty, p, st);
-    default: return launch_gemm<BN, 64>(ta, tb, td, tl2, ty, p, st);
+    case 0: return launch_gemm<BN, 0, MLP>(ta, tb, td, tl2, ty, p, st);
+    case 16: return launch_gemm<BN, 16, MLP>(ta, tb, td, tl2, ty, p, st);
+    case 32: return launch_gemm<BN, 32, MLP>(ta, tb, td, tl2, ty, p, st);
+    default: return launch_gemm<BN, 64, MLP>(ta, tb, td, tl2, ty, p, st);
   }
 }
 
@@ -390,7 +390,8 @@ svdq_status gemm_int4_impl(const uint8_t* x_codes, const uint8_t* x_scales, cons
 }
 
 svdq_status quantize_act_impl(const uint16_t* X, int M, const svdq_weight* w, uint8_t* x_codes,
-                              uint8_t* x_scales, uint16_t* D, cudaStream_t st) {
+                              uint8_t* x_scales, uint16_t* D, cudaStream_t st, float* zero_ptr = nullptr,
+                              int zero_count = 0) {
   if (w->format == SVDQ_FORMAT_INT4) return quantize_act_int4_impl(X, M, w, x_codes, x_scales, D, st);
   const int K = w->K, r = w->r, rp = r_pad_of(r);
   CUtensorMap tx{};
@@ -409,6 +410,8 @@ svdq_status quantize_act_impl(const uint16_t* X, int M, const svdq_weight* w, ui
   p.r = r;
   p.M_pad = m_pad_of(M);
   p.ks = act_k_split(M, K);
+  p.zero_ptr = zero_ptr;
+  p.zero_count = zero_count;
   switch (rp) {
     case 0: return launch_act<0>(tx, p, st);
     case 16: return launch_act<16>(tx, p, st);
@@ -418,8 +421,11 @@ svdq_status quantize_act_impl(const uint16_t* X, int M, const svdq_weight* w, ui
 }
 
 // head_dim == 0: Y row-major M x N; else Y head-major [N / head_dim][M][head_dim]
+// `mlp` (optional): the MLP epilogue's fields (inv_lambda_next ... h_out);
+// the kernel then writes the down-projection's input instead of Y.
 svdq_status gemm_impl(const uint8_t* x_codes, const uint8_t* x_scales, const uint16_t* D, int M,
-                      const svdq_weight* w, uint16_t* Y, cudaStream_t st, int head_dim = 0) {
+                      const svdq_weight* w, uint16_t* Y, cudaStream_t st, int head_dim = 0,
+                      const GemmParams* mlp = nullptr) {
   if (w->format == SVDQ_FORMAT_INT4) return gemm_int4_impl(x_codes, x_scales, D, M, w, Y, st, head_dim);
   const int N = w->N, K = w->K, r = w->r, rp = r_pad_of(r);
   const int m_tiles = (M + GEMM_BM - 1) / GEMM_BM;
@@ -437,12 +443,14 @@ svdq_status gemm_impl(const uint8_t* x_codes, const uint8_t* x_scales, const uin
   s = make_tmap(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->w_codes, K / 2, N, K / 2, 128, BN,
                 CU_TENSOR_MAP_SWIZZLE_128B);
   if (s != SVDQ_OK) return s;
-  if (head_dim == 0)
-    s = make_tmap(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, N, M, static_cast<uint64_t>(N) * 2, 16, 32,
-                  CU_TENSOR_MAP_SWIZZLE_32B);
-  else
-    s = make_tmap_heads(&ty, Y, head_dim, M, N / head_dim);
-  if (s != SVDQ_OK) return s;
+  if (mlp == nullptr) {
+    if (head_dim == 0)
+      s = make_tmap(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, N, M, static_cast<uint64_t>(N) * 2, 16, 32,
+                    CU_TENSOR_MAP_SWIZZLE_32B);
+    else
+      s = make_tmap_heads(&ty, Y, head_dim, M, N / head_dim);
+    if (s != SVDQ_OK) return s;
+  }
   if (r > 0) {
     s = make_tmap(&td, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, D, r, M, static_cast<uint64_t>(r) * 2, rp,
                   GEMM_BM, lr_swizzle(rp));
@@ -466,8 +474,44 @@ svdq_status gemm_impl(const uint8_t* x_codes, const uint8_t* x_scales, const uin
   p.n_tiles = N / BN;
   p.num_tiles = p.m_tiles * p.n_tiles;
   p.kblocks = K / GEMM_BK;
+  if (mlp != nullptr) {
+    p.inv_lambda_next = mlp->inv_lambda_next;
+    p.L1f_next = mlp->L1f_next;
+    p.r_next = mlp->r_next;
+    p.h_codes = mlp->h_codes;
+    p.h_scales = mlp->h_scales;
+    p.d_acc = mlp->d_acc;
+    p.h_out = mlp->h_out;
+    return BN == 256 ? dispatch_gemm_r<256, true>(rp, ta, tb, td, tl2, ty, p, st)
+                     : dispatch_gemm_r<128, true>(rp, ta, tb, td, tl2, ty, p, st);
+  }
   return BN == 256 ? dispatch_gemm_r<256>(rp, ta, tb, td, tl2, ty, p, st)
                    : dispatch_gemm_r<128>(rp, ta, tb, td, tl2, ty, p, st);
+}
+
+// D = bf16(acc) for the MLP pair's down-projection (M x r values), launched as
+// a programmatic dependent of the up-projection GEMM that accumulates acc.
+__global__ void d_round_kernel(const float* __restrict__ acc, uint16_t* __restrict__ D, int n) {
+  pdl_wait();
+  pdl_launch_dependents();
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
+    D[i] = static_cast<uint16_t>(pack_bf16x2(__ldcg(acc + i), 0.0f) & 0xFFFFu);
+}
+
+svdq_status launch_d_round(const float* acc, uint16_t* D, int n, cudaStream_t st) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(std::max(1, std::min((n + 255) / 256, num_sms() * 2))));
+  cfg.blockDim = dim3(256);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, d_round_kernel, acc, D, n);
+  if (e != cudaSuccess) return cuda_fail(e, "d_round_kernel launch");
+  SVDQ_CHECK_LAUNCH("d_round_kernel");
+  return SVDQ_OK;
 }
 
 // ---- few-token path (small_m.cuh) ----------------------------------------
@@ -673,6 +717,51 @@ svdq_status forward_impl(const uint16_t* X, int M, const svdq_weight* w, uint16_
   svdq_status s = quantize_act_impl(X, M, w, a.codes, a.scales, a.D, st);
   if (s != SVDQ_OK) return s;
   return gemm_impl(a.codes, a.scales, a.D, M, w, Y, st, head_dim);
+}
+
+// Workspace of the MLP pair: the up-projection's activation workspace, the
+// down-projection's (its codes, scales and D, written by the up-projection's
+// epilogue and the rounding kernel), then the float32 accumulator of D.
+struct MlpWs {
+  ActWs up, down;
+  float* d_acc;
+};
+
+size_t mlp_ws_layout(int M, int K, int F, int r_up, int r_down, uint8_t* base, MlpWs* out) {
+  const size_t a = align_up(forward_ws_bytes(M, K, r_up), kAlign);
+  const size_t b = align_up(forward_ws_bytes(M, F, r_down), kAlign);
+  const size_t c = align_up(static_cast<size_t>(M) * r_down * 4, kAlign);
+  if (out != nullptr) {
+    act_ws_layout(M, K, r_up, base, &out->up);
+    act_ws_layout(M, F, r_down, base + a, &out->down);
+    out->d_acc = reinterpret_cast<float*>(base + a + b);
+  }
+  return a + b + c;
+}
+
+svdq_status mlp_forward_impl(const uint16_t* X, int M, const svdq_weight* up, const svdq_weight* down,
+                             uint16_t* Y, uint16_t* H_out, void* ws, cudaStream_t st) {
+  MlpWs m;
+  mlp_ws_layout(M, up->K, up->N, up->r, down->r, static_cast<uint8_t*>(ws), &m);
+  const int nd = M * down->r;
+  // the up-projection's activation kernel, which also clears the D accumulator
+  svdq_status s = quantize_act_impl(X, M, up, m.up.codes, m.up.scales, m.up.D, st, m.d_acc, nd);
+  if (s != SVDQ_OK) return s;
+  GemmParams e{};
+  e.inv_lambda_next = down->inv_lambda;
+  e.L1f_next = reinterpret_cast<const uint32_t*>(down->L1f);
+  e.r_next = down->r;
+  e.h_codes = m.down.codes;
+  e.h_scales = m.down.scales;
+  e.d_acc = m.d_acc;
+  e.h_out = H_out;
+  s = gemm_impl(m.up.codes, m.up.scales, m.up.D, M, up, nullptr, st, 0, &e);
+  if (s != SVDQ_OK) return s;
+  if (down->r > 0) {
+    s = launch_d_round(m.d_acc, m.down.D, nd, st);
+    if (s != SVDQ_OK) return s;
+  }
+  return gemm_impl(m.down.codes, m.down.scales, m.down.D, M, down, Y, st);
 }
 
 struct PrepWs {
@@ -1243,6 +1332,32 @@ svdq_status svdq_linear_forward_noalloc(const uint16_t* X, int M, const svdq_wei
   s = noalloc_scratch_address(&scratch);
   if (s != SVDQ_OK) return s;
   return forward_impl(X, M, w, Y, scratch, static_cast<cudaStream_t>(stream), 0);
+}
+
+size_t svdq_mlp_workspace_bytes(int M, int K, int F, int N, int r_up, int r_down) {
+  if (M < 0 || check_layer_shape(F, K, r_up) != SVDQ_OK || check_layer_shape(N, F, r_down) != SVDQ_OK ||
+      r_down > 32)
+    return 0;
+  return mlp_ws_layout(M, K, F, r_up, r_down, nullptr, nullptr);
+}
+
+svdq_status svdq_mlp_forward(const uint16_t* X, int M, const svdq_weight* up, const svdq_weight* down, uint16_t* Y,
+                             uint16_t* H_out, void* ws, size_t ws_bytes, void* stream) {
+  svdq_status s = check_weight(up);
+  if (s != SVDQ_OK) return s;
+  s = check_weight(down);
+  if (s != SVDQ_OK) return s;
+  if (up->format != SVDQ_FORMAT_NVFP4 || down->format != SVDQ_FORMAT_NVFP4 || down->K != up->N)
+    return SVDQ_ERR_INVALID_ARG;
+  if (down->r > 32) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  if (M < 0) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  if (X == nullptr || Y == nullptr || ws == nullptr) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(Y) || !aligned16(ws) || (H_out != nullptr && !aligned16(H_out)))
+    return SVDQ_ERR_MISALIGNED;
+  if (ws_bytes < mlp_ws_layout(M, up->K, up->N, up->r, down->r, nullptr, nullptr))
+    return SVDQ_ERR_WORKSPACE_TOO_SMALL;
+  return mlp_forward_impl(X, M, up, down, Y, H_out, ws, static_cast<cudaStream_t>(stream));
 }
 
 svdq_status svdq_weight_export(const svdq_weight* w, uint8_t* host_codes, uint8_t* host_scales,
