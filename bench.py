@@ -258,6 +258,84 @@ def _time_steps(step, flush, steps, warmup, st):
     return [a.elapsed_time(b) for a, b in ev]
 
 
+def _l2_bytes():
+    import torch
+    try:
+        return int(torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size)
+    except Exception:
+        return 126 << 20
+
+
+class LayerCopies:
+    """`n` independent copies of one prepared layer (weight buffer, input,
+    output, workspace), so that consecutive steps touch different memory and
+    the steps' inputs together exceed L2 (a copy of the weight is a plain
+    device copy of the prepared buffer, bound again)."""
+
+    def __init__(self, lin, X, M, n):
+        import torch
+        import w4a4_rank_corrected_act_b200 as svdq
+        self.M, self.N, self.K = M, lin.N, lin.K
+        nb = lin.workspace_bytes(M)
+        self.nb = nb
+        self.items = []
+        for i in range(n):
+            if i == 0:
+                buf, w, Xi = lin.buf, lin.w, X
+            else:
+                buf = lin.buf.clone()
+                w = svdq.svdq_weight_bind_format(buf.data_ptr(), buf.numel(), lin.N, lin.K, lin.r,
+                                                 int(lin.has_bias), svdq.FORMAT_NAMES[lin.format])
+                Xi = X.clone()
+            Yi = torch.empty((M, lin.N), dtype=torch.int16, device="cuda")
+            wsi = torch.empty(max(nb, 256), dtype=torch.uint8, device="cuda")
+            self.items.append((buf, w, Xi, Yi, wsi))
+
+    @staticmethod
+    def count(footprint_bytes, lo=2, hi=16):
+        """Copies whose footprints together exceed twice the L2 cache."""
+        return int(min(hi, max(lo, -(-2 * _l2_bytes() // max(footprint_bytes, 1)))))
+
+    def step(self, i, sh):
+        import w4a4_rank_corrected_act_b200 as svdq
+        _, w, X, Y, ws = self.items[i % len(self.items)]
+        svdq.svdq_linear_forward(X.data_ptr(), self.M, w, Y.data_ptr(), ws.data_ptr(), self.nb, sh)
+
+
+def time_back_to_back(step, steps, warmup, st):
+    """Device time (ms) of `steps` calls step(i) issued back to back on `st`,
+    the sequence captured once in a CUDA graph and replayed (so that host
+    launch overhead does not pace the GPU); falls back to eager launches if
+    capture fails.  Returns (total_ms, graph_used)."""
+    import torch
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    g = None
+    try:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=st):
+            for i in range(steps):
+                step(i)
+        g.replay()
+        torch.cuda.synchronize()
+    except Exception:
+        g = None
+        torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(st)
+    if g is not None:
+        g.replay()
+    else:
+        for i in range(steps):
+            step(i)
+    b.record(st)
+    torch.cuda.synchronize()
+    used = g is not None
+    del g
+    return a.elapsed_time(b), used
+
+
 def layer_entry(spec, step_ms):
     """Per-workload entry of the bench line: layer latency percentiles, 4-bit
     TFLOP/s and roofline fractions.  Below the ridge (few tokens) the layer
@@ -291,8 +369,10 @@ def layer_entry(spec, step_ms):
 
 
 def measure_configs(names, steps, warmup, st, flush):
-    """Each named workload as one svdq_linear_forward per step (L2 flushed
-    between steps), on its own seeded inputs; weights prepared untimed."""
+    """Each named workload as one svdq_linear_forward per step on its own
+    seeded inputs (weights prepared untimed): `steps` steps back to back over
+    rotating copies (inputs beyond L2; the per-layer figure), and the same
+    layer alone with L2 flushed before it (the isolated latency)."""
     import torch
     import w4a4_rank_corrected_act_b200 as svdq
     from workloads import gen
@@ -304,16 +384,55 @@ def measure_configs(names, steps, warmup, st, flush):
         dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()  # noqa: E731
         lin = svdq.SvdqLinear(dev(d["W"]), torch.from_numpy(d["lam"]).cuda(), dev(d["bias"]), r=spec.r)
         X = dev(d["X"])
-        Y = torch.empty((spec.M, spec.N), dtype=torch.int16, device="cuda")
-        nb = lin.workspace_bytes(spec.M)
-        ws = torch.empty(max(nb, 256), dtype=torch.uint8, device="cuda")
-
-        def step():
-            svdq.svdq_linear_forward(X.data_ptr(), spec.M, lin.w, Y.data_ptr(), ws.data_ptr(), nb, sh)
-
-        out[name] = layer_entry(spec, _time_steps(step, flush, steps, warmup, st))
-        del lin, X, Y, ws
+        foot = X.numel() * 2 + lin.buf.numel() + lin.workspace_bytes(spec.M) + spec.M * spec.N * 2
+        cp = LayerCopies(lin, X, spec.M, LayerCopies.count(foot))
+        total_ms, graph = time_back_to_back(lambda i: cp.step(i, sh), steps, warmup, st)
+        iso = _time_steps(lambda: cp.step(0, sh), flush, steps, warmup, st)
+        e = layer_entry(spec, [total_ms / steps])
+        e.update({"copies": len(cp.items), "graph": graph,
+                  "us_isolated_p50": round(float(np.percentile(iso, 50)) * 1e3, 2)})
+        out[name] = e
+        del lin, X, cp
         torch.cuda.empty_cache()
+    return out
+
+
+def measure_mlp_pair(steps, warmup, st, flush):
+    """The MLP pair at 1024 x 1024 (up 3072 -> 12288, GELU, down 12288 -> 3072,
+    M = 4608, r = 32) through svdq_mlp_forward: back to back over rotating
+    copies, and alone with L2 flushed.  The down-projection's smoothing
+    factors come from its own input recipe (GELU of a normal draw)."""
+    import torch
+    import w4a4_rank_corrected_act_b200 as svdq
+    from workloads import gen
+    sh = int(st.cuda_stream)
+    su, sd = gen.workload("mlp_up"), gen.workload("mlp_down")
+    du, dd = gen.make_linear(su), gen.make_linear(sd)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()  # noqa: E731
+    up = svdq.SvdqLinear(dev(du["W"]), torch.from_numpy(du["lam"]).cuda(), dev(du["bias"]), r=su.r)
+    down = svdq.SvdqLinear(dev(dd["W"]), torch.from_numpy(dd["lam"]).cuda(), dev(dd["bias"]), r=sd.r)
+    M, K, F, N = su.M, su.K, su.N, sd.N
+    nb = svdq.svdq_mlp_workspace_bytes(M, K, F, N, su.r, sd.r)
+    X = dev(du["X"])
+    copies = []
+    for i in range(2):
+        copies.append((X if i == 0 else X.clone(), torch.empty((M, N), dtype=torch.int16, device="cuda"),
+                       torch.empty(nb, dtype=torch.uint8, device="cuda")))
+
+    def step(i):
+        Xi, Yi, wsi = copies[i % len(copies)]
+        svdq.svdq_mlp_forward(Xi.data_ptr(), M, up.w, down.w, Yi.data_ptr(), 0, wsi.data_ptr(), nb, sh)
+
+    total_ms, graph = time_back_to_back(step, steps, warmup, st)
+    iso = _time_steps(lambda: step(0), flush, steps, warmup, st)
+    flops = 2.0 * M * K * F + 2.0 * M * F * N
+    us = total_ms / steps * 1e3
+    out = {"M": M, "K": K, "F": F, "N": N, "r": su.r, "us_per_pair": round(us, 2),
+           "tflops": round(flops / (us * 1e-6) / 1e12, 1),
+           "us_isolated_p50": round(float(np.percentile(iso, 50)) * 1e3, 2), "graph": graph,
+           "kernels_per_pair": 4 if sd.r else 3}
+    del up, down, copies
+    torch.cuda.empty_cache()
     return out
 
 
@@ -337,7 +456,9 @@ def run_native(args):
     spec = gen.workload(args.workload)
     M, K, N, r = spec.M, spec.K, spec.N, spec.r
     d = gen.make_linear(spec)
-    st = torch.cuda.current_stream()
+    # a stream of our own (the legacy default stream cannot be captured in a graph)
+    st = torch.cuda.Stream()
+    torch.cuda.set_stream(st)
     sh = int(st.cuda_stream)
 
     def dev(a):
@@ -347,39 +468,63 @@ def run_native(args):
     lin = svdq.SvdqLinear(dev(d["W"]), torch.from_numpy(d["lam"]).cuda(), dev(d["bias"]), r=r,
                           format=args.format)
     X = dev(d["X"])
-    Y = torch.empty((M, N), dtype=torch.int16, device="cuda")
     nb = lin.workspace_bytes(M)
-    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    # consecutive steps use different copies of the weight, input, output and
+    # workspace, whose footprints together exceed twice the L2 cache
+    foot = X.numel() * 2 + lin.buf.numel() + nb + M * N * 2
+    cp = LayerCopies(lin, X, M, LayerCopies.count(foot))
+    _, _, _, Y, ws = cp.items[0]
 
-    def step():
-        svdq.svdq_linear_forward(X.data_ptr(), M, lin.w, Y.data_ptr(), ws.data_ptr(), nb, sh)
+    def step_i(i):
+        cp.step(i, sh)
 
-    for _ in range(args.warmup):
-        flush.zero_()
-        step()
+    for i in range(args.warmup):
+        step_i(i)
     torch.cuda.synchronize()
     svdq.svdq_clear_device_status(sh)
+    # the K timed steps, captured once as one CUDA graph (host launch overhead
+    # would otherwise pace the GPU for the shorter layers)
+    graph = None
+    try:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=st):
+            for i in range(args.steps):
+                step_i(i)
+    except Exception:
+        graph = None
+    torch.cuda.synchronize()
 
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    def timed_steps():
+        if graph is not None:
+            graph.replay()
+        else:
+            for i in range(args.steps):
+                step_i(i)
+
+    def load_for(seconds):
+        t0 = time.perf_counter()
+        while time.perf_counter() - t0 < seconds:
+            timed_steps()
+            torch.cuda.synchronize()
+
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         # the sampler sees >= 0.5 s of this workload before and after the timed steps
-        _run_for(0.5, flush, step)
+        load_for(0.5)
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
-        for i in range(args.steps):
-            flush.zero_()
-            starts[i].record(st)
-            step()
-            ends[i].record(st)
+        t_start.record(st)
+        timed_steps()
+        t_end.record(st)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
-        _run_for(0.5, flush, step)
-    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = max_over_ranks(sum(step_ms), device="cuda")
+        load_for(0.5)
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end), device="cuda")
+    # the same layer alone, L2 flushed before each step (latency of one isolated call)
+    step_ms = _time_steps(lambda: step_i(0), flush, args.steps, args.warmup, st)
     status = svdq.svdq_get_device_status(sh)
     if status:
         raise SystemExit(f"device status word {status:#x}: a kernel gave up a wait")
@@ -441,16 +586,20 @@ def run_native(args):
         # every workload of the benchmark set, one layer each (the qkv entry
         # repeats the headline's own steps), the small-token layer against
         # HBM, and one DiT block of four linears
-        configs = {"qkv": layer_entry(spec, step_ms)}
+        configs = {"qkv": layer_entry(spec, [ms_per_step])}
+        configs["qkv"].update({"copies": len(cp.items), "graph": graph is not None,
+                               "us_isolated_p50": round(float(np.percentile(step_ms, 50)) * 1e3, 2)})
         configs.update(measure_configs(["small", "mlp_up", "mlp_down", "small_m"], args.steps, args.warmup,
                                        st, flush))
         configs["mlp_pair_unfused"] = {
             "us": round(configs["mlp_up"]["us_per_layer"] + configs["mlp_down"]["us_per_layer"], 2),
             "note": "up- and down-projection timed as separate layers (GELU between them not included)"}
-        b_ms, b_layers, b_flops, b_tokens = measure_block("b1", args.steps, args.warmup, st, flush)
-        b_p50 = float(np.percentile(b_ms, 50))
-        configs["block_b1"] = {"tokens": b_tokens, "us_per_block": round(b_p50 * 1e3, 2),
-                               "tflops": round(b_flops / (b_p50 * 1e-3) / 1e12, 1), "layers_us": b_layers}
+        configs["mlp_pair_fused"] = measure_mlp_pair(args.steps, args.warmup, st, flush)
+        b_ms, b_layers, b_flops, b_tokens, b_b2b = measure_block("b1", args.steps, args.warmup, st, flush)
+        configs["block_b1"] = {"tokens": b_tokens, "us_per_block": round(b_b2b * 1e3, 2),
+                               "tflops": round(b_flops / (b_b2b * 1e-3) / 1e12, 1),
+                               "us_isolated_p50": round(float(np.percentile(b_ms, 50)) * 1e3, 2),
+                               "layers_us_isolated": b_layers}
         if svdq.svdq_get_device_status(sh):
             raise SystemExit("a kernel gave up a wait")
 
@@ -465,13 +614,17 @@ def run_native(args):
             "config": {"workload": f"{spec.name}: DiT joint-attention QKV projection at 1024x1024"
                                    if spec.name == "qkv" else spec.name,
                        "M": M, "K": K, "N": N, "r": r, "bias": True, "format": args.format,
-                       "l2": "flushed between steps (256 MiB write outside the step events)",
+                       "l2": f"steps back to back over {len(cp.items)} copies of weight, input, output and "
+                             f"workspace ({len(cp.items) * foot / 2**20:.0f} MiB > 2 x L2), no flush; "
+                             "isolated latencies flushed (256 MiB write before each step)",
+                       "timing": ("the K steps captured as one CUDA graph, replayed between two events"
+                                  if graph is not None else "K eager launches between two events"),
                        "parallelism": f"replicas x{world} (token-parallel, no collective)"},
             "pct_fp4_peak": {"of_spec_9000": round(value / FP4_SPEC_TFLOPS, 4),
                              "of_measured_bf16x4": round(value / fp4_peak, 4)} if not int4 else None,
             "us_per_layer": round(ms_per_step * 1e3, 2),
-            "step_us_percentiles": {"p50": round(float(np.percentile(step_ms, 50)) * 1e3, 2),
-                                    "p95": round(float(np.percentile(step_ms, 95)) * 1e3, 2)},
+            "isolated_step_us_percentiles": {"p50": round(float(np.percentile(step_ms, 50)) * 1e3, 2),
+                                             "p95": round(float(np.percentile(step_ms, 95)) * 1e3, 2)},
             "roofline": roofline,
             "kernels": {"act_quant": act},
             "e2e": e2e,
@@ -532,11 +685,13 @@ def measure_block(tag, steps, warmup, st, flush):
     step_ms = [e[0].elapsed_time(e[-1]) for e in per]
     layer_us = {spec.name: round(statistics.mean(e[j].elapsed_time(e[j + 1]) for e in per) * 1e3, 2)
                 for j, (spec, *_) in enumerate(layers)}
+    # the blocks back to back (their footprint exceeds L2 on its own), as one graph
+    b2b_ms, graph = time_back_to_back(lambda i: step(), steps, warmup, st)
     flops = sum(2.0 * spec.M * spec.N * spec.K for spec, *_ in layers)
     tokens = layers[0][0].M
     del layers
     torch.cuda.empty_cache()
-    return step_ms, layer_us, flops, tokens
+    return step_ms, layer_us, flops, tokens, b2b_ms / steps
 
 
 def run_block(args):
@@ -545,13 +700,14 @@ def run_block(args):
     import w4a4_rank_corrected_act_b200 as svdq
 
     torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
-    st = torch.cuda.current_stream()
+    st = torch.cuda.Stream()
+    torch.cuda.set_stream(st)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
     with ClockSampler(0) as clk:
-        step_ms, layer_us, flops, tokens = measure_block(args.block, args.steps, args.warmup, st, flush)
+        step_ms, layer_us, flops, tokens, b2b_ms = measure_block(args.block, args.steps, args.warmup, st, flush)
     if svdq.svdq_get_device_status(int(st.cuda_stream)):
         raise SystemExit("a kernel gave up a wait")
-    total_ms = sum(step_ms)
+    total_ms = b2b_ms * args.steps
     out = {
         "metric": METRIC + " (DiT block: four linears)", "value": round(flops * args.steps / (total_ms * 1e-3) / 1e12, 2),
         "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
@@ -559,9 +715,10 @@ def run_block(args):
         "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic (seeded DiT-shaped inputs; no checkpoint)",
         "config": {"workload": f"DiT block, {tokens} tokens: QKV 3072->9216, out 3072->3072, "
                                "up 3072->12288, down 12288->3072, r=32, bias",
-                   "l2": "flushed between steps (256 MiB write outside the step events)",
+                   "l2": "blocks back to back (a block's footprint exceeds L2), one CUDA graph; "
+                         "per-layer times from isolated blocks with L2 flushed before each",
                    "parallelism": "replicas x1 (token-parallel, no collective)"},
-        "layers_us": layer_us,
+        "layers_us_isolated": layer_us,
         "step_us_percentiles": {"p50": round(float(np.percentile(step_ms, 50)) * 1e3, 2),
                                 "p95": round(float(np.percentile(step_ms, 95)) * 1e3, 2)},
         "gpu_launches": 8 * args.steps,
