@@ -68,12 +68,19 @@ struct GemmParams {
 
 constexpr int GEMM_MLP_THREADS = 512;   // 4 + 8 epilogue + 4 scale warps
 
-template <int BN>
+template <int BN, bool MLP = false>
 struct GemmCfg {
   static constexpr uint32_t kBTile = BN * 128;
   static constexpr uint32_t kSFBTile = (BN / 128) * GEMM_SFA_TILE;
   static constexpr uint32_t kStage = GEMM_A_TILE + kBTile + GEMM_SFA_TILE + kSFBTile;
-  static constexpr int kStages = (BN == 256 ? 4 : 6);
+  // the MLP epilogue, not the mainloop, bounds that kernel: one ring stage
+  // fewer leaves room for its per-tile constants
+  static constexpr int kStages = (BN == 256 ? 4 : 6) - (MLP ? 1 : 0);
+  // MLP epilogue constants of one tile (two slots): 1/lambda of the next layer,
+  // the bias (bf16), and the next layer's L1 fragments for the tile's BN / 16 k-steps
+  // (r_next <= 32: at most 4 column tiles of 256 bytes each per k-step)
+  static constexpr uint32_t kConstInv = BN * 4, kConstBias = BN * 2, kConstL1 = (BN / 16) * 4 * 256;
+  static constexpr uint32_t kConstSlot = MLP ? kConstBias + kConstInv + kConstL1 : 0;
   static constexpr uint32_t kTmemCols = 512;
   // tensor-memory columns: two scale buffers in the top 96, accumulators below
   static constexpr uint32_t kSfaCol0 = 416;              // + 16 j: 4 k-blocks x 4 columns
@@ -81,8 +88,8 @@ struct GemmCfg {
   static constexpr uint32_t kAcc1Col = (BN == 256 ? 160 : 128);
   static constexpr int kOverlapChunks = (BN == 256 ? (256 - 160) / 32 : 0);
   static constexpr uint32_t kOutBytes = 4 * GEMM_STAGE_OUT;   // epilogue staging, 4 warps
-  static constexpr uint32_t kBarBytes = (2 * kStages + 9) * 8 + 16;
-  static constexpr uint32_t kSmemBytes = kStages * kStage + kOutBytes + kBarBytes + 1024;
+  static constexpr uint32_t kBarBytes = (2 * kStages + 13) * 8 + 16;
+  static constexpr uint32_t kSmemBytes = kStages * kStage + kOutBytes + 2 * kConstSlot + kBarBytes + 1024;
   static_assert(kSfbCol0 + 32 + 4 * (BN / 32) <= kTmemCols, "scale columns");
   static_assert(kAcc1Col + BN <= kSfaCol0, "accumulator buffer 1");
   static_assert(kStage % 1024 == 0, "stage alignment");
@@ -272,38 +279,60 @@ __device__ __forceinline__ void epilogue_tile(uint32_t acc, uint32_t lane_addr, 
 }
 
 // GELU, tanh form, y/2 (1 + tanh u) with u = sqrt(2/pi) (y + 0.044715 y^3),
-// evaluated as y / (1 + e^{-2u}) (the same function: 1 + tanh u = 2 / (1 +
-// e^{-2u})), which keeps its relative accuracy where 1 + tanh u cancels, with
-// the device's exponential and reciprocal.  Where e^{-2u} > e^80 the value is
-// y e^{2u} to float32 precision, taken with the exponential that keeps
-// subnormal results (the value is a subnormal number below about y = -10).
-__device__ __forceinline__ float gelu_tanh_f32(float y) {
-  const float y3 = y * y * y;
-  const float m2u = -1.5957691216057308f * fmaf(0.044715f, y3, y);   // -2u
-  if (m2u > 80.0f) return y * expf(-m2u);
+// evaluated without cancellation through 1 + tanh u = 2 / (1 + e^{-2u}):
+// with e = e^{-|2u|} <= 1,  GELU(y) = y / (1 + e) for u >= 0 and
+// y e / (1 + e) for u < 0.  e is taken as e^{64 ln 2 - |2u|} 2^-64 with the
+// device's exponential, so that where it is tiny (y below about -10) it
+// becomes a subnormal number instead of being flushed, and the result y e
+// keeps its subnormal value.  No branch: one exponential and one reciprocal
+// per element.
+__device__ __forceinline__ float gelu_tail_f32(float y, float two_u) {
+  const float e = __expf(44.361419555836500f - fabsf(two_u)) * 0x1p-64f;
   float rc;
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(rc) : "f"(1.0f + __expf(m2u)));
-  return y * rc;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(rc) : "f"(1.0f + e));
+  return (two_u < 0.0f ? y * e : y) * rc;
 }
 
-// MLP epilogue of one 16-column piece of the up-projection's tile for the
-// warp owning rows row0 .. row0 + 31 (lane = row): columns n .. n + 15 of the
-// hidden layer.  For each element: Y_up = bf16(acc + bias); H = bf16(GELU(Y_up));
-// Hhat = f32(H / lambda_next).  The 16 Hhat of the row are one NVFP4 block of
-// the down-projection's input: its 8 code bytes and its scale go straight to
-// that layer's activation buffers.  bf16(Hhat) goes through a per-warp
-// 32 x 16 shared tile into two m16n8k16 A fragments, whose bf16 MMAs with the
-// piece's 16 rows of L1_next accumulate the tile's partial of D_next in dacc.
+// The same for a pair (packed f32x2 for the polynomial 2u = 2 sqrt(2/pi) (y +
+// 0.044715 y^3)); returns the two results packed as bf16 (RNE), lo first.
+__device__ __forceinline__ uint32_t gelu_tanh_bf16x2(float y0, float y1) {
+  const uint64_t y = f32x2_pack(y0, y1);
+  const uint64_t y2 = f32x2_mul(y, y);
+  const uint64_t t = f32x2_fma(f32x2_mul(y2, y), f32x2_pack(0.044715f, 0.044715f), y);
+  float u0, u1;
+  f32x2_unpack(f32x2_mul(t, f32x2_pack(1.5957691216057308f, 1.5957691216057308f)), u0, u1);
+  return pack_bf16x2(gelu_tail_f32(y0, u0), gelu_tail_f32(y1, u1));
+}
+
+// The MLP epilogue's per-tile constants in shared memory: 1/lambda_next of
+// the tile's columns, its bias (bf16; null without bias) and the next layer's
+// L1 fragments of its k-steps (piece c: c * nt * 32 + t * 32 + lane).
+struct MlpTileConsts {
+  const float* inv;
+  const uint16_t* bias;
+  const uint2* l1f;
+};
+
+// MLP epilogue of one 16-column piece (piece c of the tile: hidden columns
+// n .. n + 15) of the up-projection's tile for the warp owning rows row0 ..
+// row0 + 31 (lane = row).  For each element: Y_up = bf16(acc + bias);
+// H = bf16(GELU(Y_up)); Hhat = f32(H / lambda_next).  The 16 Hhat of the row
+// are one NVFP4 block of the down-projection's input: its 8 code bytes and its
+// scale go straight to that layer's activation buffers.  bf16(Hhat) goes
+// through a per-warp 32 x 16 shared tile into two m16n8k16 A fragments, whose
+// bf16 MMAs with the piece's 16 rows of L1_next accumulate the tile's partial
+// of D_next in dacc.
 template <int NT>
-__device__ __forceinline__ void mlp_piece(const uint32_t (&v)[16], int n, int row, const GemmParams& p,
-                                          uint8_t* dstage, uint32_t dstage_u, int lane, float (&dacc)[2][NT][4],
-                                          uint64_t six, uint64_t neg_y6) {
+__device__ __forceinline__ void mlp_piece(const uint32_t (&v)[16], int c, int n, int row, const GemmParams& p,
+                                          const MlpTileConsts& tc, uint8_t* dstage, uint32_t dstage_u, int lane,
+                                          float (&dacc)[2][NT][4], uint64_t six, uint64_t neg_y6) {
   const int F = p.N;
   // bias and 1/lambda_next of the piece: the same 16 values on every lane
+  // (shared-memory broadcasts)
   float b[16];
-  if (p.bias != nullptr) {
-    const uint4 b0 = __ldg(reinterpret_cast<const uint4*>(p.bias + n));
-    const uint4 b1 = __ldg(reinterpret_cast<const uint4*>(p.bias + n + 8));
+  if (tc.bias != nullptr) {
+    const uint4 b0 = reinterpret_cast<const uint4*>(tc.bias + 16 * c)[0];
+    const uint4 b1 = reinterpret_cast<const uint4*>(tc.bias + 16 * c)[1];
     const uint32_t bw[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -317,7 +346,7 @@ __device__ __forceinline__ void mlp_piece(const uint32_t (&v)[16], int n, int ro
   float inv[16];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const float4 x = __ldg(reinterpret_cast<const float4*>(p.inv_lambda_next + n) + i);
+    const float4 x = reinterpret_cast<const float4*>(tc.inv + 16 * c)[i];
     inv[4 * i] = x.x; inv[4 * i + 1] = x.y; inv[4 * i + 2] = x.z; inv[4 * i + 3] = x.w;
   }
   uint32_t hb[8];          // H, packed bf16 pairs
@@ -325,7 +354,7 @@ __device__ __forceinline__ void mlp_piece(const uint32_t (&v)[16], int n, int ro
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const uint32_t yb = pack_bf16x2(__uint_as_float(v[2 * i]) + b[2 * i], __uint_as_float(v[2 * i + 1]) + b[2 * i + 1]);
-    const uint32_t h = pack_bf16x2(gelu_tanh_f32(bf16_bits_to_f32(yb & 0xFFFFu)), gelu_tanh_f32(bf16_bits_to_f32(yb >> 16)));
+    const uint32_t h = gelu_tanh_bf16x2(bf16_bits_to_f32(yb & 0xFFFFu), bf16_bits_to_f32(yb >> 16));
     hb[i] = h;
     nh[i] = f32x2_mul(f32x2_pack(bf16_bits_to_f32(h & 0xFFFFu), bf16_bits_to_f32(h >> 16)),
                       f32x2_pack(-inv[2 * i], -inv[2 * i + 1]));
@@ -343,6 +372,7 @@ __device__ __forceinline__ void mlp_piece(const uint32_t (&v)[16], int n, int ro
   // rows of the last row tile at and beyond M get zero scales (padding)
   p.h_scales[sf_offset(static_cast<uint32_t>(row), static_cast<uint32_t>(n / 16), static_cast<uint32_t>(F))] =
       static_cast<uint8_t>(row < p.M ? sc : 0u);
+  if (p.r_next == 0) return;
   // bf16(Hhat) = -bf16(-Hhat) (rounding commutes with negation)
   uint32_t a8[8];
 #pragma unroll
@@ -360,11 +390,10 @@ __device__ __forceinline__ void mlp_piece(const uint32_t (&v)[16], int n, int ro
   for (int mt = 0; mt < 2; ++mt)
     ldmatrix_x4(dstage_u + (16 * mt + (lane & 15)) * 32 + (lane >> 4) * 16, a[mt][0], a[mt][1], a[mt][2], a[mt][3]);
   const int nt = p.r_next >> 3;
-  const uint2* f = reinterpret_cast<const uint2*>(p.L1f_next);
 #pragma unroll
   for (int t = 0; t < NT; ++t) {
     if (t < nt) {
-      const uint2 bf = __ldg(f + ((static_cast<size_t>(n / 16) * nt + t) * 32 + lane));
+      const uint2 bf = tc.l1f[(c * nt + t) * 32 + lane];
 #pragma unroll
       for (int mt = 0; mt < 2; ++mt) mma_bf16_16816(dacc[mt][t], a[mt][0], a[mt][1], a[mt][2], a[mt][3], bf.x, bf.y);
     }
@@ -377,8 +406,8 @@ __device__ __forceinline__ void mlp_piece(const uint32_t (&v)[16], int n, int ro
 // batched read), then the tile's partial D_next into d_acc.
 template <int BN, int KOV, typename Order, typename Release>
 __device__ __forceinline__ void mlp_epilogue_tile(uint32_t acc, uint32_t lane_addr, int lane, int half, int row0,
-                                                  int n0, const GemmParams& p, uint8_t* dstage, uint32_t dstage_u,
-                                                  Order order, Release release) {
+                                                  int n0, const GemmParams& p, const MlpTileConsts& tc,
+                                                  uint8_t* dstage, uint32_t dstage_u, Order order, Release release) {
   constexpr int kMine = BN / 32, kOvMine = KOV / 2, kNT = 4;
   const int row = row0 + lane;
   const uint64_t six = f32x2_pack(6.0f, 6.0f);
@@ -399,17 +428,20 @@ __device__ __forceinline__ void mlp_epilogue_tile(uint32_t acc, uint32_t lane_ad
     tc_fence_before();
     release();
 #pragma unroll
-    for (int j = 0; j < kOvMine; ++j)
-      mlp_piece<kNT>(ov[j], n0 + 16 * order(half + 2 * j), row, p, dstage, dstage_u, lane, dacc, six, neg_y6);
+    for (int j = 0; j < kOvMine; ++j) {
+      const int c = order(half + 2 * j);
+      mlp_piece<kNT>(ov[j], c, n0 + 16 * c, row, p, tc, dstage, dstage_u, lane, dacc, six, neg_y6);
+    }
   } else {
     tc_fence_before();
     release();
   }
   for (int j = kOvMine; j < kMine; ++j) {
     uint32_t v[16];
-    tmem_ld_32x32b_x16(acc + lane_addr + order(half + 2 * j) * 16, v);
+    const int c = order(half + 2 * j);
+    tmem_ld_32x32b_x16(acc + lane_addr + c * 16, v);
     tmem_ld_wait();
-    mlp_piece<kNT>(v, n0 + 16 * order(half + 2 * j), row, p, dstage, dstage_u, lane, dacc, six, neg_y6);
+    mlp_piece<kNT>(v, c, n0 + 16 * c, row, p, tc, dstage, dstage_u, lane, dacc, six, neg_y6);
   }
   // the tile's partial D_next: fragment rows lane / 4 (+ 8) of each 16-row
   // block, columns 8 t + 2 (lane % 4) (+ 1)
@@ -436,7 +468,7 @@ __global__ void __launch_bounds__(MLP ? GEMM_MLP_THREADS : GEMM_THREADS, 1)
     fp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                     const __grid_constant__ CUtensorMap tm_d, const __grid_constant__ CUtensorMap tm_l2,
                     const __grid_constant__ CUtensorMap tm_y, const GemmParams p) {
-  using Cfg = GemmCfg<BN>;
+  using Cfg = GemmCfg<BN, MLP>;
   constexpr int S = Cfg::kStages;
   constexpr uint32_t kLRLayout = (R_PAD == 64 ? LAYOUT_SW128 : R_PAD == 32 ? LAYOUT_SW64 : LAYOUT_SW32);
   constexpr uint32_t kLRSbo = 8 * R_PAD * 2;
@@ -449,11 +481,13 @@ __global__ void __launch_bounds__(MLP ? GEMM_MLP_THREADS : GEMM_THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* out_stage = smem + S * Cfg::kStage;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(out_stage + Cfg::kOutBytes);
+  uint8_t* const_slots = out_stage + Cfg::kOutBytes;   // MLP epilogue constants, 2 slots
+  uint64_t* bars = reinterpret_cast<uint64_t*>(const_slots + 2 * Cfg::kConstSlot);
   // bars[0..S) full, [S..2S) empty, 2S/2S+1 tmem_full[2], 2S+2 tmem_free, 2S+3 drain,
   // 2S+4/2S+5 sf_ready[2] (scale warps -> MMA), 2S+6/2S+7 sf_free[2] (MMA -> scale warps),
-  // 2S+8 tmem_done (tensor memory no longer used: MMA thread + epilogue warps)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 9);
+  // 2S+8 tmem_done (tensor memory no longer used: MMA thread + epilogue warps),
+  // 2S+9/2S+10 const_full[2], 2S+11/2S+12 const_free[2] (MLP epilogue constants)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 13);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -472,6 +506,8 @@ __global__ void __launch_bounds__(MLP ? GEMM_MLP_THREADS : GEMM_THREADS, 1)
   auto sf_ready = [&](uint32_t b) { return smem_u32(bars + 2 * S + 4 + b); };
   auto sf_free = [&](uint32_t b) { return smem_u32(bars + 2 * S + 6 + b); };
   const uint32_t tmem_done = smem_u32(bars + 2 * S + 8);
+  auto const_full = [&](int b) { return smem_u32(bars + 2 * S + 9 + b); };
+  auto const_free = [&](int b) { return smem_u32(bars + 2 * S + 11 + b); };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -487,6 +523,10 @@ __global__ void __launch_bounds__(MLP ? GEMM_MLP_THREADS : GEMM_THREADS, 1)
       mbar_init(sf_free(b), 1);
     }
     mbar_init(tmem_done, kEpiWarps + 1);   // the MMA thread and the epilogue warps
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(const_full(b), 1);
+      mbar_init(const_free(b), kEpiWarps);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -557,9 +597,32 @@ __global__ void __launch_bounds__(MLP ? GEMM_MLP_THREADS : GEMM_THREADS, 1)
         }
       };
       bool ok = true;
-      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+      int const_parity[2] = {-1, -1};
+      int local_t = 0;
+      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x, ++local_t) {
         const int mb = t % p.m_tiles, nb = t / p.m_tiles;
         const int m0 = mb * GEMM_BM, n0 = nb * BN;
+        if constexpr (MLP) {
+          // the MLP epilogue's constants of this tile into slot local_t % 2,
+          // once the epilogue has finished the tile that used it before
+          const int cb = local_t & 1;
+          if (local_t >= 2 &&
+              !mbar_wait(const_free(cb), static_cast<uint32_t>((local_t >> 1) - 1) & 1u, abort_flag, KID_GEMM, 3)) {
+            ok = false;
+            break;
+          }
+          const uint32_t slot = smem_u32(const_slots + cb * Cfg::kConstSlot);
+          const int nt = p.r_next >> 3;
+          const uint32_t l1_bytes = static_cast<uint32_t>(BN / 16) * nt * 256u;
+          mbar_arrive_expect_tx(const_full(cb), Cfg::kConstInv + (p.bias != nullptr ? Cfg::kConstBias : 0u) + l1_bytes);
+          bulk_load(slot, p.inv_lambda_next + n0, Cfg::kConstInv, const_full(cb));
+          if (p.bias != nullptr) bulk_load(slot + Cfg::kConstInv, p.bias + n0, Cfg::kConstBias, const_full(cb));
+          if (l1_bytes > 0)
+            bulk_load(slot + Cfg::kConstInv + Cfg::kConstBias,
+                      reinterpret_cast<const uint8_t*>(p.L1f_next) + static_cast<size_t>(n0 / 16) * nt * 256u, l1_bytes,
+                      const_full(cb));
+          const_parity[cb] = (local_t >> 1) & 1;
+        }
         if (R_PAD > 0) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1, abort_flag, KID_GEMM, 1)) { ok = false; break; }
           mbar_arrive_expect_tx(full_bar(stage), tx_lr);
@@ -587,6 +650,8 @@ __global__ void __launch_bounds__(MLP ? GEMM_MLP_THREADS : GEMM_THREADS, 1)
       if (*abort_flag) {
         for (int s = 0; s < S; ++s)
           if (fill_parity[s] >= 0) mbar_wait_drain(full_bar(s), static_cast<uint32_t>(fill_parity[s]));
+        for (int b = 0; b < 2; ++b)
+          if (const_parity[b] >= 0) mbar_wait_drain(const_full(b), static_cast<uint32_t>(const_parity[b]));
       }
     }
   } else if (warp == 1) {
@@ -669,6 +734,7 @@ __global__ void __launch_bounds__(MLP ? GEMM_MLP_THREADS : GEMM_THREADS, 1)
       const int m0 = mb * GEMM_BM, n0 = nb * BN;
       const int buf = local & 1;
       const uint32_t acc = tmem_base + (buf ? Cfg::kAcc1Col : 0u);
+      if (!mbar_wait(const_full(buf), static_cast<uint32_t>(local >> 1) & 1u, abort_flag, KID_GEMM, 10)) break;
       if (!mbar_wait(tmem_full(buf), static_cast<uint32_t>(local >> 1) & 1u, abort_flag, KID_GEMM, 8)) break;
       tc_fence_after();
       constexpr int kPieces = BN / 16, kOv = 2 * Cfg::kOverlapChunks;
@@ -677,7 +743,14 @@ __global__ void __launch_bounds__(MLP ? GEMM_MLP_THREADS : GEMM_THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(tmem_free);
       };
-      mlp_epilogue_tile<BN, kOv>(acc, lane_addr, lane, half, m0 + q * 32, n0, p, dstage, dstage_u, order, release);
+      const uint8_t* cs = const_slots + buf * Cfg::kConstSlot;
+      const MlpTileConsts tc{reinterpret_cast<const float*>(cs),
+                             p.bias != nullptr ? reinterpret_cast<const uint16_t*>(cs + Cfg::kConstInv) : nullptr,
+                             reinterpret_cast<const uint2*>(cs + Cfg::kConstInv + Cfg::kConstBias)};
+      mlp_epilogue_tile<BN, kOv>(acc, lane_addr, lane, half, m0 + q * 32, n0, p, tc, dstage, dstage_u, order,
+                                 release);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(const_free(buf));
     }
     // this warp's tensor-memory reads are over (every tcgen05.ld waited)
     tc_fence_before();

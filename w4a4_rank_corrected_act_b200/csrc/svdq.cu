@@ -252,7 +252,7 @@ template <int BN, int R_PAD, bool MLP = false>
 svdq_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
                         const CUtensorMap& tl2, const CUtensorMap& ty, const GemmParams& p,
                         cudaStream_t st) {
-  using Cfg = GemmCfg<BN>;
+  using Cfg = GemmCfg<BN, MLP>;
   {
     const svdq_status so = opt_in_smem(reinterpret_cast<const void*>(fp4_gemm_kernel<BN, R_PAD, MLP>),
                                        Cfg::kSmemBytes, "cudaFuncSetAttribute(gemm)");
