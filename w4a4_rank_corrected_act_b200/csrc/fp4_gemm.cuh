@@ -66,7 +66,8 @@ struct GemmParams {
   uint16_t* h_out;                // optional M x F bf16: H itself (null: not written)
 };
 
-constexpr int GEMM_MLP_THREADS = 512;   // 4 + 8 epilogue + 4 scale warps
+constexpr int GEMM_MLP_PARTS = 2;       // MLP epilogue warps per lane quarter
+constexpr int GEMM_MLP_THREADS = 32 * (4 + 4 * GEMM_MLP_PARTS + 4);   // 4 + 8 epilogue + 4 scale warps
 
 template <int BN, bool MLP = false>
 struct GemmCfg {
@@ -87,7 +88,8 @@ struct GemmCfg {
   static constexpr uint32_t kSfbCol0 = 448;              // + 32 j: 4 k-blocks x BN/32 columns
   static constexpr uint32_t kAcc1Col = (BN == 256 ? 160 : 128);
   static constexpr int kOverlapChunks = (BN == 256 ? (256 - 160) / 32 : 0);
-  static constexpr uint32_t kOutBytes = 4 * GEMM_STAGE_OUT;   // epilogue staging, 4 warps
+  // epilogue staging: 4 warps x two pieces, or 1 KB per MLP epilogue warp
+  static constexpr uint32_t kOutBytes = MLP ? 4 * GEMM_MLP_PARTS * 1024 : 4 * GEMM_STAGE_OUT;
   static constexpr uint32_t kBarBytes = (2 * kStages + 13) * 8 + 16;
   static constexpr uint32_t kSmemBytes = kStages * kStage + kOutBytes + 2 * kConstSlot + kBarBytes + 1024;
   static_assert(kSfbCol0 + 32 + 4 * (BN / 32) <= kTmemCols, "scale columns");
@@ -400,15 +402,17 @@ __device__ __forceinline__ void mlp_piece(const uint32_t (&v)[16], int c, int n,
   }
 }
 
-// MLP epilogue of one 128 x BN tile for one of the two warps of lane quarter
-// q (half h takes the pieces order(h), order(h + 2), ...; the first of them
-// are the columns the next tile's accumulator shares, released after one
-// batched read), then the tile's partial D_next into d_acc.
+// MLP epilogue of one 128 x BN tile for one of the GEMM_MLP_PARTS warps of
+// lane quarter q (part h takes the pieces order(h), order(h + PARTS), ...; the
+// first KOV pieces are the columns the next tile's accumulator shares,
+// released after one batched read), then the tile's partial D_next into d_acc.
 template <int BN, int KOV, typename Order, typename Release>
-__device__ __forceinline__ void mlp_epilogue_tile(uint32_t acc, uint32_t lane_addr, int lane, int half, int row0,
+__device__ __forceinline__ void mlp_epilogue_tile(uint32_t acc, uint32_t lane_addr, int lane, int part, int row0,
                                                   int n0, const GemmParams& p, const MlpTileConsts& tc,
                                                   uint8_t* dstage, uint32_t dstage_u, Order order, Release release) {
-  constexpr int kMine = BN / 32, kOvMine = KOV / 2, kNT = 4;
+  constexpr int kPieces = BN / 16, kParts = GEMM_MLP_PARTS, kNT = 4;
+  static_assert(KOV % kParts == 0, "every part takes the same number of shared pieces");
+  constexpr int kOvMine = KOV / kParts;
   const int row = row0 + lane;
   const uint64_t six = f32x2_pack(6.0f, 6.0f);
   const float y6 = e4m3_table_entry(0x4C).y;   // code 0x4C is 6.0: RN(1/6)
@@ -423,22 +427,22 @@ __device__ __forceinline__ void mlp_epilogue_tile(uint32_t acc, uint32_t lane_ad
   if constexpr (kOvMine > 0) {
     uint32_t ov[kOvMine][16];
 #pragma unroll
-    for (int j = 0; j < kOvMine; ++j) tmem_ld_32x32b_x16(acc + lane_addr + order(half + 2 * j) * 16, ov[j]);
+    for (int j = 0; j < kOvMine; ++j) tmem_ld_32x32b_x16(acc + lane_addr + order(part + kParts * j) * 16, ov[j]);
     tmem_ld_wait();
     tc_fence_before();
     release();
 #pragma unroll
     for (int j = 0; j < kOvMine; ++j) {
-      const int c = order(half + 2 * j);
+      const int c = order(part + kParts * j);
       mlp_piece<kNT>(ov[j], c, n0 + 16 * c, row, p, tc, dstage, dstage_u, lane, dacc, six, neg_y6);
     }
   } else {
     tc_fence_before();
     release();
   }
-  for (int j = kOvMine; j < kMine; ++j) {
+  for (int i = part + KOV; i < kPieces; i += kParts) {
     uint32_t v[16];
-    const int c = order(half + 2 * j);
+    const int c = order(i);
     tmem_ld_32x32b_x16(acc + lane_addr + c * 16, v);
     tmem_ld_wait();
     mlp_piece<kNT>(v, c, n0 + 16 * c, row, p, tc, dstage, dstage_u, lane, dacc, six, neg_y6);
@@ -472,9 +476,10 @@ __global__ void __launch_bounds__(MLP ? GEMM_MLP_THREADS : GEMM_THREADS, 1)
   constexpr int S = Cfg::kStages;
   constexpr uint32_t kLRLayout = (R_PAD == 64 ? LAYOUT_SW128 : R_PAD == 32 ? LAYOUT_SW64 : LAYOUT_SW32);
   constexpr uint32_t kLRSbo = 8 * R_PAD * 2;
-  // epilogue warps: 4 (one per lane quarter), or 8 for the MLP epilogue (two
-  // per lane quarter, splitting the tile's columns); the scale warps follow
-  constexpr int kEpiWarps = MLP ? 8 : 4;
+  // epilogue warps: 4 (one per lane quarter), or 4 * GEMM_MLP_PARTS for the
+  // MLP epilogue (that many per lane quarter, splitting the tile's columns);
+  // the scale warps follow
+  constexpr int kEpiWarps = MLP ? 4 * GEMM_MLP_PARTS : 4;
   constexpr int kScaleWarp0 = 4 + kEpiWarps;
 
   extern __shared__ uint8_t smem_raw[];
@@ -724,7 +729,7 @@ __global__ void __launch_bounds__(MLP ? GEMM_MLP_THREADS : GEMM_THREADS, 1)
     }
   } else if (MLP && warp >= 4 && warp < kScaleWarp0) {
     // --------------------------------------------------------- MLP epilogue
-    const int q = warp & 3, half = (warp - 4) >> 2;
+    const int q = warp & 3, part = (warp - 4) >> 2;
     uint8_t* dstage = out_stage + (warp - 4) * 1024;
     const uint32_t dstage_u = smem_u32(dstage);
     const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
@@ -747,7 +752,7 @@ __global__ void __launch_bounds__(MLP ? GEMM_MLP_THREADS : GEMM_THREADS, 1)
       const MlpTileConsts tc{reinterpret_cast<const float*>(cs),
                              p.bias != nullptr ? reinterpret_cast<const uint16_t*>(cs + Cfg::kConstInv) : nullptr,
                              reinterpret_cast<const uint2*>(cs + Cfg::kConstInv + Cfg::kConstBias)};
-      mlp_epilogue_tile<BN, kOv>(acc, lane_addr, lane, half, m0 + q * 32, n0, p, tc, dstage, dstage_u, order,
+      mlp_epilogue_tile<BN, kOv>(acc, lane_addr, lane, part, m0 + q * 32, n0, p, tc, dstage, dstage_u, order,
                                  release);
       __syncwarp();
       if (lane == 0) mbar_arrive(const_free(buf));
