@@ -90,8 +90,10 @@ struct GemmCfg {
   static constexpr int kOverlapChunks = (BN == 256 ? (256 - 160) / 32 : 0);
   // epilogue staging: 4 warps x two pieces, or 1 KB per MLP epilogue warp
   static constexpr uint32_t kOutBytes = MLP ? 4 * GEMM_MLP_PARTS * 1024 : 4 * GEMM_STAGE_OUT;
+  static constexpr uint32_t kTabBytes = MLP ? 128 * 8 : 0;   // E4M3 (s, RN(1/s)) for the MLP epilogue
   static constexpr uint32_t kBarBytes = (2 * kStages + 13) * 8 + 16;
-  static constexpr uint32_t kSmemBytes = kStages * kStage + kOutBytes + 2 * kConstSlot + kBarBytes + 1024;
+  static constexpr uint32_t kSmemBytes =
+      kStages * kStage + kOutBytes + 2 * kConstSlot + kTabBytes + kBarBytes + 1024;
   static_assert(kSfbCol0 + 32 + 4 * (BN / 32) <= kTmemCols, "scale columns");
   static_assert(kAcc1Col + BN <= kSfaCol0, "accumulator buffer 1");
   static_assert(kStage % 1024 == 0, "stage alignment");
@@ -283,36 +285,40 @@ __device__ __forceinline__ void epilogue_tile(uint32_t acc, uint32_t lane_addr, 
 // GELU, tanh form, y/2 (1 + tanh u) with u = sqrt(2/pi) (y + 0.044715 y^3),
 // evaluated without cancellation through 1 + tanh u = 2 / (1 + e^{-2u}):
 // with e = e^{-|2u|} <= 1,  GELU(y) = y / (1 + e) for u >= 0 and
-// y e / (1 + e) for u < 0.  e is taken as e^{64 ln 2 - |2u|} 2^-64 with the
-// device's exponential, so that where it is tiny (y below about -10) it
-// becomes a subnormal number instead of being flushed, and the result y e
-// keeps its subnormal value.  No branch: one exponential and one reciprocal
-// per element.
-__device__ __forceinline__ float gelu_tail_f32(float y, float two_u) {
-  const float e = __expf(44.361419555836500f - fabsf(two_u)) * 0x1p-64f;
-  float rc;
+// y e / (1 + e) for u < 0.  With t = 2u log2(e), e = 2^-|t|, taken as
+// 2^(64 - |t|) 2^-64 with the device's base-2 exponential, so that where it is
+// tiny (y below about -10) it becomes a subnormal number instead of being
+// flushed, and the result y e keeps its subnormal value.  No branch: one
+// exponential and one reciprocal per element.
+__device__ __forceinline__ float gelu_tail_f32(float y, float t) {
+  float p, rc;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(p) : "f"(64.0f - fabsf(t)));
+  const float e = p * 0x1p-64f;
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(rc) : "f"(1.0f + e));
-  return (two_u < 0.0f ? y * e : y) * rc;
+  return (t < 0.0f ? y * e : y) * rc;
 }
 
-// The same for a pair (packed f32x2 for the polynomial 2u = 2 sqrt(2/pi) (y +
-// 0.044715 y^3)); returns the two results packed as bf16 (RNE), lo first.
+// The same for a pair, the polynomial t = 2 sqrt(2/pi) log2(e) (y + 0.044715
+// y^3) in packed f32x2; returns the two results packed as bf16 (RNE), lo first.
 __device__ __forceinline__ uint32_t gelu_tanh_bf16x2(float y0, float y1) {
+  constexpr float kC = 2.302208198144325f;          // 2 sqrt(2/pi) log2(e)
+  constexpr float kC3 = 0.1029432395800235f;        // kC * 0.044715
   const uint64_t y = f32x2_pack(y0, y1);
-  const uint64_t y2 = f32x2_mul(y, y);
-  const uint64_t t = f32x2_fma(f32x2_mul(y2, y), f32x2_pack(0.044715f, 0.044715f), y);
-  float u0, u1;
-  f32x2_unpack(f32x2_mul(t, f32x2_pack(1.5957691216057308f, 1.5957691216057308f)), u0, u1);
-  return pack_bf16x2(gelu_tail_f32(y0, u0), gelu_tail_f32(y1, u1));
+  const uint64_t p = f32x2_fma(f32x2_mul(y, y), f32x2_pack(kC3, kC3), f32x2_pack(kC, kC));
+  float t0, t1;
+  f32x2_unpack(f32x2_mul(y, p), t0, t1);
+  return pack_bf16x2(gelu_tail_f32(y0, t0), gelu_tail_f32(y1, t1));
 }
 
 // The MLP epilogue's per-tile constants in shared memory: 1/lambda_next of
 // the tile's columns, its bias (bf16; null without bias) and the next layer's
-// L1 fragments of its k-steps (piece c: c * nt * 32 + t * 32 + lane).
+// L1 fragments of its k-steps (piece c: c * nt * 32 + t * 32 + lane); and the
+// kernel's table of E4M3 scales (s, RN(1/s)).
 struct MlpTileConsts {
   const float* inv;
   const uint16_t* bias;
   const uint2* l1f;
+  const float2* tab;
 };
 
 // MLP epilogue of one 16-column piece (piece c of the tile: hidden columns
@@ -362,7 +368,7 @@ __device__ __forceinline__ void mlp_piece(const uint32_t (&v)[16], int c, int n,
                       f32x2_pack(-inv[2 * i], -inv[2 * i + 1]));
   }
   uint32_t sc;
-  const uint64_t codes = nvfp4_quant_block16_x2(nh, six, neg_y6, sc);
+  const uint64_t codes = nvfp4_quant_block16_x2(nh, tc.tab, six, neg_y6, sc);
   if (row < p.M) {
     *reinterpret_cast<uint64_t*>(p.h_codes + static_cast<size_t>(row) * (F / 2) + n / 2) = codes;
     if (p.h_out != nullptr) {
@@ -375,13 +381,15 @@ __device__ __forceinline__ void mlp_piece(const uint32_t (&v)[16], int c, int n,
   p.h_scales[sf_offset(static_cast<uint32_t>(row), static_cast<uint32_t>(n / 16), static_cast<uint32_t>(F))] =
       static_cast<uint8_t>(row < p.M ? sc : 0u);
   if (p.r_next == 0) return;
-  // bf16(Hhat) = -bf16(-Hhat) (rounding commutes with negation)
+  // the fragments hold bf16(-Hhat) = -bf16(Hhat) (rounding commutes with
+  // negation): dacc accumulates the negated partial, negated back when it is
+  // added to d_acc
   uint32_t a8[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     float lo, hi;
     f32x2_unpack(nh[i], lo, hi);
-    a8[i] = pack_bf16x2(lo, hi) ^ 0x80008000u;
+    a8[i] = pack_bf16x2(lo, hi);
   }
   __syncwarp();   // the previous piece's fragments have been read
   *reinterpret_cast<uint4*>(dstage + lane * 32) = make_uint4(a8[0], a8[1], a8[2], a8[3]);
@@ -415,7 +423,7 @@ __device__ __forceinline__ void mlp_epilogue_tile(uint32_t acc, uint32_t lane_ad
   constexpr int kOvMine = KOV / kParts;
   const int row = row0 + lane;
   const uint64_t six = f32x2_pack(6.0f, 6.0f);
-  const float y6 = e4m3_table_entry(0x4C).y;   // code 0x4C is 6.0: RN(1/6)
+  const float y6 = tc.tab[0x4C].y;   // code 0x4C is 6.0: RN(1/6)
   const uint64_t neg_y6 = f32x2_pack(-y6, -y6);
   float dacc[2][kNT][4];
 #pragma unroll
@@ -457,12 +465,12 @@ __device__ __forceinline__ void mlp_epilogue_tile(uint32_t acc, uint32_t lane_ad
       if (t >= nt) continue;
       const int r_lo = row0 + 16 * mt + (lane >> 2), col = 8 * t + 2 * (lane & 3);
       if (r_lo < p.M) {
-        atomicAdd(p.d_acc + static_cast<size_t>(r_lo) * p.r_next + col, dacc[mt][t][0]);
-        atomicAdd(p.d_acc + static_cast<size_t>(r_lo) * p.r_next + col + 1, dacc[mt][t][1]);
+        atomicAdd(p.d_acc + static_cast<size_t>(r_lo) * p.r_next + col, -dacc[mt][t][0]);
+        atomicAdd(p.d_acc + static_cast<size_t>(r_lo) * p.r_next + col + 1, -dacc[mt][t][1]);
       }
       if (r_lo + 8 < p.M) {
-        atomicAdd(p.d_acc + static_cast<size_t>(r_lo + 8) * p.r_next + col, dacc[mt][t][2]);
-        atomicAdd(p.d_acc + static_cast<size_t>(r_lo + 8) * p.r_next + col + 1, dacc[mt][t][3]);
+        atomicAdd(p.d_acc + static_cast<size_t>(r_lo + 8) * p.r_next + col, -dacc[mt][t][2]);
+        atomicAdd(p.d_acc + static_cast<size_t>(r_lo + 8) * p.r_next + col + 1, -dacc[mt][t][3]);
       }
     }
 }
@@ -487,7 +495,8 @@ __global__ void __launch_bounds__(MLP ? GEMM_MLP_THREADS : GEMM_THREADS, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* out_stage = smem + S * Cfg::kStage;
   uint8_t* const_slots = out_stage + Cfg::kOutBytes;   // MLP epilogue constants, 2 slots
-  uint64_t* bars = reinterpret_cast<uint64_t*>(const_slots + 2 * Cfg::kConstSlot);
+  float2* e4m3_tab = reinterpret_cast<float2*>(const_slots + 2 * Cfg::kConstSlot);   // MLP epilogue only
+  uint64_t* bars = reinterpret_cast<uint64_t*>(const_slots + 2 * Cfg::kConstSlot + Cfg::kTabBytes);
   // bars[0..S) full, [S..2S) empty, 2S/2S+1 tmem_full[2], 2S+2 tmem_free, 2S+3 drain,
   // 2S+4/2S+5 sf_ready[2] (scale warps -> MMA), 2S+6/2S+7 sf_free[2] (MMA -> scale warps),
   // 2S+8 tmem_done (tensor memory no longer used: MMA thread + epilogue warps),
@@ -538,6 +547,9 @@ __global__ void __launch_bounds__(MLP ? GEMM_MLP_THREADS : GEMM_THREADS, 1)
   if (warp == 2) {
     tmem_alloc(smem_u32(tmem_slot), Cfg::kTmemCols);
     tmem_relinquish();
+  }
+  if constexpr (MLP) {
+    for (int c = threadIdx.x; c < 128; c += blockDim.x) e4m3_tab[c] = e4m3_table_entry(c);
   }
   tc_fence_before();
   __syncthreads();
@@ -751,7 +763,7 @@ __global__ void __launch_bounds__(MLP ? GEMM_MLP_THREADS : GEMM_THREADS, 1)
       const uint8_t* cs = const_slots + buf * Cfg::kConstSlot;
       const MlpTileConsts tc{reinterpret_cast<const float*>(cs),
                              p.bias != nullptr ? reinterpret_cast<const uint16_t*>(cs + Cfg::kConstInv) : nullptr,
-                             reinterpret_cast<const uint2*>(cs + Cfg::kConstInv + Cfg::kConstBias)};
+                             reinterpret_cast<const uint2*>(cs + Cfg::kConstInv + Cfg::kConstBias), e4m3_tab};
       mlp_epilogue_tile<BN, kOv>(acc, lane_addr, lane, part, m0 + q * 32, n0, p, tc, dstage, dstage_u, order,
                                  release);
       __syncwarp();

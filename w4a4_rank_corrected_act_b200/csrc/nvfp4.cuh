@@ -186,23 +186,30 @@ __device__ __forceinline__ uint32_t nvfp4_quant_half_block_x2(const uint64_t (&n
 
 // One whole 16-element block in one thread: the same result as
 // nvfp4_quant_half_block_x2 for the pair of lanes holding its halves, for the
-// 16 values given NEGATED and packed in pairs (nv[u] = (-v[2u], -v[2u+1])).
-// s and RN(1/s) are formed in place (e4m3_table_entry) instead of read from a
-// table.  Returns the 16 codes, element 0 in the lowest nibble.
-__device__ __forceinline__ uint64_t nvfp4_quant_block16_x2(const uint64_t (&nv)[8], uint64_t six, uint64_t neg_y6,
-                                                          uint32_t& scale_code) {
-  float am = 0.0f;
+// 16 values given NEGATED and packed in pairs (nv[u] = (-v[2u], -v[2u+1])),
+// with s and RN(1/s) read from `tab` (the 128 entries of e4m3_table_entry,
+// in shared memory).  The block maximum is taken as a tree (max is exact, so
+// the order does not matter).  Returns the 16 codes, element 0 in the lowest
+// nibble.
+__device__ __forceinline__ uint64_t nvfp4_quant_block16_x2(const uint64_t (&nv)[8], const float2* tab, uint64_t six,
+                                                          uint64_t neg_y6, uint32_t& scale_code) {
+  float m[8];
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
     float lo, hi;
     f32x2_unpack(nv[u], lo, hi);
-    am = fmaxf(am, fmaxf(fabsf(lo), fabsf(hi)));
+    m[u] = fmaxf(fabsf(lo), fabsf(hi));
   }
+#pragma unroll
+  for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+    for (int u = 0; u < w; ++u) m[u] = fmaxf(m[u], m[u + w]);
+  const float am = m[0];
   float a6, a6b;
   f32x2_unpack(quotient_f32x2(f32x2_pack(-am, -am), six, neg_y6), a6, a6b);   // RN(amax / 6)
   const uint32_t sc = e4m3_rn_satfinite(a6);
   scale_code = sc;
-  const float2 sy = e4m3_table_entry(sc);
+  const float2 sy = tab[sc];
   const uint64_t s2 = f32x2_pack(sy.x, sy.x), neg_y2 = f32x2_pack(-sy.y, -sy.y);
   uint64_t q0[4], q1[4];
 #pragma unroll
