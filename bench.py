@@ -442,6 +442,23 @@ def measure_mlp_pair(steps, warmup, st, flush):
     return out
 
 
+def run_mlp_pair(args):
+    """--mlp-pair: the fused MLP pair alone (svdq_mlp_forward), one JSON line."""
+    import torch
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    st = torch.cuda.Stream()
+    torch.cuda.set_stream(st)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    pair = measure_mlp_pair(args.steps, args.warmup, st, flush)
+    print(json.dumps({"metric": "SVDQ W4A4 MLP pair (up, GELU, down) TFLOP/s", "value": pair["tflops"],
+                      "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+                      "higher_is_better": True, "dtype": "nvfp4", "data": "synthetic",
+                      "config": {"workload": "mlp pair at 1024x1024", "M": pair["M"], "K": pair["K"],
+                                 "F": pair["F"], "N": pair["N"], "r": pair["r"]},
+                      "mlp_pair_fused": pair}), flush=True)
+    return 0
+
+
 def run_native(args):
     import torch
     import torch.distributed as dist
@@ -872,6 +889,8 @@ def main(argv=None):
     ap.add_argument("--block", choices=["b1", "b4"], default=None,
                     help="time the four linears of a DiT block (QKV, out, up, down) back to back "
                          "on one stream (b1: 4608 tokens, b4: 18432) instead of one workload")
+    ap.add_argument("--mlp-pair", action="store_true",
+                    help="time only the fused MLP pair (svdq_mlp_forward) at 1024x1024")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -881,6 +900,8 @@ def main(argv=None):
         args.cpu_baseline = False
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
         raise SystemExit("for --gpus > 1 launch with torch.distributed.run (one rank per GPU)")
+    if args.mlp_pair:
+        return run_mlp_pair(args)
     if args.block:
         if args.format != "nvfp4":
             raise SystemExit("--block times the NVFP4 layer")

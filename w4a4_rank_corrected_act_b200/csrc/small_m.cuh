@@ -448,7 +448,8 @@ __global__ void __launch_bounds__(SMALL_THREADS, 2)
         uint8_t* dt = smem + p.off_d;
         constexpr int kMaxSlices = SMALL_MAX_K / SMALL_ACT_COLS;
         for (int e = q * 32 + lane; e < TN * R_PAD; e += 128) {
-          const int t = e / R_PAD, j = e % R_PAD;
+          constexpr int kRp = R_PAD > 0 ? R_PAD : 1;   // (this branch runs only with R_PAD > 0)
+          const int t = e / kRp, j = e % kRp;
           float v = 0.0f;
           if (t < p.M && j < p.r) {
             // all slices' partials are loaded first (one round trip), then
