@@ -87,3 +87,17 @@ def test_kernel_rooflines_for_the_three_regimes():
     for entry in (g, a):
         t = entry["traffic"]
         assert t is None or t > 0
+
+
+def test_few_token_roofline_is_one_layer_call_against_hbm():
+    peaks, _ = bench._peaks()
+    e = bench.few_token_roofline(16, 18432, 3072, 32, 0.0132, "small_m")
+    # X, the weight's codes and scales, L1, L2, 1/lambda, bias and Y, each once
+    alg = 16 * 3072 * 2 + 18432 * 3072 // 2 + 18432 * 3072 // 16 + 3072 * 32 * 2 + 18432 * 32 * 2 \
+        + 3072 * 4 + 18432 * 2 + 16 * 18432 * 2
+    assert e["algorithmic_bytes_per_launch"] == alg == 33964032
+    assert e["bound"] == "hbm" and e["unit"] == "GB/s" and e["peak"] == peaks["hbm_gbs"]
+    assert e["achieved"] == pytest.approx(alg / 13.2e-6 / 1e9, rel=1e-3)
+    assert e["frac"] == pytest.approx(e["achieved"] / e["peak"], rel=1e-3)
+    t = e["traffic"]
+    assert t is None or t > 0
