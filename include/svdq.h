@@ -95,6 +95,10 @@ typedef enum svdq_status {
  *   L2t        N x r bf16, L2^T = V_r.
  *   inv_lambda K float32, f32(1 / lambda).
  *   bias       N bf16, or NULL when has_bias == 0.
+ *   L1t        r x K bf16, L1 transposed (row j holds L1[:, j]; read by the
+ *              layer's activation kernel, whose tensor-core product with the
+ *              activation tile needs L1 with K contiguous).  Written, like
+ *              L1f, by svdq_prepare_weight and svdq_weight_import.
  *
  * INT4 format (format == SVDQ_FORMAT_INT4): the other 4-bit format of the
  * layer, used before Blackwell (chaosnode.de "Nunchaku Lite", section
@@ -120,6 +124,7 @@ typedef struct svdq_weight {
   uint16_t* L2t;
   float* inv_lambda;
   uint16_t* bias;
+  uint16_t* L1t;
 } svdq_weight;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -145,7 +150,10 @@ size_t svdq_act_scales_bytes(int M, int K);
 
 /* Workspace of svdq_linear_forward (and its host, head-major and no-allocation
  * variants), 256-byte aligned fields.  For the general path: codes (M x K/2),
- * scales (tile layout above) and D (M x r bf16).  For M <= 32 and K <= 3840
+ * scales (tile layout above) and D (M x r bf16), then, for r > 0, the
+ * activation kernel's K-split partials of D (float32, 8 roundup(M,128) r)
+ * and their flags (uint64 [roundup(M,128)/128][8]; see svdq_quantize_act_ws;
+ * their contents need not be initialised).  For M <= 32 and K <= 3840
  * the few-token path (see svdq_linear_forward) uses, from the start of the
  * same buffer: codes M x K/2; the scale words uint32 [K/64][32] (word j of
  * token m holds the E4M3 codes of its 16-element blocks 4 j .. 4 j + 3, low
@@ -214,6 +222,22 @@ svdq_status svdq_prepare_weight(const uint16_t* W, const float* lambda, const ui
  * ------------------------------------------------------------------------- */
 svdq_status svdq_quantize_act(const uint16_t* X, int M, const svdq_weight* w, uint8_t* x_codes,
                               uint8_t* x_scales, uint16_t* D, void* stream);
+
+/* The same outputs through the activation kernel that svdq_linear_forward
+ * runs: for r > 0 and enough work per CTA (each of the 128-row CTAs, K split
+ * across up to 8 of them, walks at least 12 stages of 64 columns) a kernel
+ * with D on the tensor cores, which needs a workspace for the K split's
+ * float32 partials of D and their flags; otherwise svdq_quantize_act's.
+ *   ws        device, at least svdq_act_workspace_bytes(M, K, r) bytes
+ *             (256 bytes when r == 0), contents need not be initialised
+ * Codes and scales equal those of svdq_quantize_act bit for bit; D may
+ * differ from its D by float32 summation order (both are within D's bound),
+ * and equals the D that svdq_linear_forward computes for the same X.  With
+ * r == 0 or an INT4 weight this is svdq_quantize_act.  Returns 0 bytes for
+ * an invalid shape. */
+size_t svdq_act_workspace_bytes(int M, int K, int r);
+svdq_status svdq_quantize_act_ws(const uint16_t* X, int M, const svdq_weight* w, uint8_t* x_codes,
+                                 uint8_t* x_scales, uint16_t* D, void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
  * Block-scaled FP4 GEMM with the low-rank branch and bias fused:
@@ -424,6 +448,10 @@ svdq_status svdq_int4_scales_to_native(const uint16_t* logical, int rows, int ro
  *                                  (a multiple of 128)
  *   SVDQ_OVERRIDE_SMALL_M          1 = never take the few-token path of
  *                                  svdq_linear_forward (see there)
+ *   SVDQ_OVERRIDE_ACT_KERNEL       activation kernel of svdq_linear_forward
+ *                                  and svdq_quantize_act_ws for r > 0: 1 = the
+ *                                  16-row kernel, 2 = the 128-row kernel with
+ *                                  D on the tensor cores
  * Results are identical under every setting up to float32 summation order
  * (the tests check each against the oracle).  SVDQ_ERR_INVALID_ARG for an
  * unknown `which` or a negative value.
@@ -432,7 +460,8 @@ svdq_status svdq_int4_scales_to_native(const uint16_t* logical, int rows, int ro
 #define SVDQ_OVERRIDE_GEMM_BN 2
 #define SVDQ_OVERRIDE_HOST_CHUNK_ROWS 3
 #define SVDQ_OVERRIDE_SMALL_M 4
-#define SVDQ_OVERRIDE_COUNT 5
+#define SVDQ_OVERRIDE_ACT_KERNEL 5
+#define SVDQ_OVERRIDE_COUNT 6
 svdq_status svdq_set_override(int which, int value);
 
 /* Synchronise `stream` and report the device status word of the current

@@ -98,15 +98,17 @@ def y_with_d(y_oracle64: np.ndarray, d_oracle_bits: np.ndarray, d_gpu_bits: np.n
 
 def gpu_d(lin, X_dev, M: int) -> np.ndarray:
     """The activation kernel's D for X (the same kernel, deterministic, that the
-    layer's forward runs), as bf16 bits."""
+    layer's forward runs: svdq_quantize_act_ws), as bf16 bits."""
     import w4a4_rank_corrected_act_b200 as svdq
     t = torch()
     K, r = lin.K, lin.r
     codes = empty_u8(svdq.svdq_act_codes_bytes(M, K))
     scales = empty_u8(svdq.svdq_act_scales_bytes(M, K))
     D = t.empty((M, max(r, 1)), dtype=t.int16, device="cuda")
-    svdq.svdq_quantize_act(X_dev.data_ptr(), M, lin.w, codes.data_ptr(), scales.data_ptr(), D.data_ptr(),
-                           stream())
+    nb = svdq.svdq_act_workspace_bytes(M, K, r)
+    ws = empty_u8(nb)
+    svdq.svdq_quantize_act_ws(X_dev.data_ptr(), M, lin.w, codes.data_ptr(), scales.data_ptr(), D.data_ptr(),
+                              ws.data_ptr(), nb, stream())
     t.cuda.synchronize()
     return D.cpu().numpy().view(np.uint16)[:, :r]
 

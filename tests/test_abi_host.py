@@ -45,9 +45,14 @@ def test_sizes():
     assert svdq.svdq_act_scales_bytes(0, 3072) == 0
     al = lambda x: (x + 255) // 256 * 256                              # noqa: E731
     M, N, K, r = 4608, 9216, 3072, 32
-    assert svdq.svdq_forward_workspace_bytes(M, N, K, r) == al(M * K // 2) + al(M * K // 16) + al(M * r * 2)
+    mp = (M + 127) // 128 * 128
+    partials = al(8 * mp * r * 4) + al(mp // 128 * 8 * 8)
+    assert svdq.svdq_forward_workspace_bytes(M, N, K, r) == (al(M * K // 2) + al(M * K // 16) + al(M * r * 2)
+                                                             + partials)
+    assert svdq.svdq_act_workspace_bytes(M, K, r) == partials
+    assert svdq.svdq_act_workspace_bytes(M, K, 0) == 256
     wb = (al(N * K // 2) + al(N * K // 16) + al(K * r * 2) + al(K * r * 2) + al(N * r * 2)
-          + al(K * 4) + al(N * 2))
+          + al(K * 4) + al(N * 2) + al(K * r * 2))
     assert svdq.svdq_weight_bytes(N, K, r, 1) == wb
     assert svdq.svdq_weight_bytes(N, K, r, 0) == wb - al(N * 2)
 
@@ -65,17 +70,17 @@ def test_weight_bind_carves_aligned_fields():
     nbytes = svdq.svdq_weight_bytes(N, K, r, 1)
     base = 0x7F0000000000                   # never dereferenced: bind is pointer arithmetic
     w = svdq.svdq_weight_bind(base, nbytes, N, K, r, 1)
-    fields = [w.w_codes, w.w_scales, w.L1, w.L1f, w.L2t, w.inv_lambda, w.bias]
+    fields = [w.w_codes, w.w_scales, w.L1, w.L1f, w.L2t, w.inv_lambda, w.bias, w.L1t]
     assert all(f % 256 == 0 for f in fields)
     assert fields == sorted(fields) and fields[0] == base
-    assert w.bias + N * 2 <= base + nbytes
+    assert w.L1t + K * r * 2 <= base + nbytes
     assert (w.N, w.K, w.r, w.has_bias) == (N, K, r, 1)
     with pytest.raises(svdq.SvdqError, match="WORKSPACE_TOO_SMALL"):
         svdq.svdq_weight_bind(base, nbytes - 1, N, K, r, 1)
     with pytest.raises(svdq.SvdqError, match="MISALIGNED"):
         svdq.svdq_weight_bind(base + 16, nbytes, N, K, r, 1)
     w0 = svdq.svdq_weight_bind(base, svdq.svdq_weight_bytes(N, K, 0, 0), N, K, 0, 0)
-    assert w0.L1 is None and w0.bias is None
+    assert w0.L1 is None and w0.bias is None and w0.L1t is None
 
 
 def _tile_offset(row, kb16, K):

@@ -41,13 +41,16 @@ def test_full_size_sampled(name):
     _, wc, ws = ref.residual_quantize(w_hat, exp["L1"], L2s)
     assert int((wc != exp["w_codes"][wrows]).sum()) == 0
     assert np.array_equal(ws, exp["w_scales"][wrows])
-    # activations through svdq_quantize_act, then Y through svdq_linear_forward
+    # activations through the forward's own activation kernel
+    # (svdq_quantize_act_ws), then Y through svdq_linear_forward
     X = dev_u16(d["X"])
     codes = empty_u8(svdq.svdq_act_codes_bytes(M, K))
     scales = empty_u8(svdq.svdq_act_scales_bytes(M, K))
     D = t.empty((M, r), dtype=t.int16, device="cuda")
-    svdq.svdq_quantize_act(X.data_ptr(), M, lin.w, codes.data_ptr(), scales.data_ptr(),
-                           D.data_ptr(), stream())
+    nb = svdq.svdq_act_workspace_bytes(M, K, r)
+    wsb = empty_u8(nb)
+    svdq.svdq_quantize_act_ws(X.data_ptr(), M, lin.w, codes.data_ptr(), scales.data_ptr(),
+                              D.data_ptr(), wsb.data_ptr(), nb, stream())
     Y = lin.forward(X.view(t.bfloat16))
     t.cuda.synchronize()
     rows = _sample(M, 64, 2)

@@ -57,6 +57,7 @@ def _weight_with(K, N, r, inv_lambda, L1=None, has_bias=False):
     if r:
         put(w.L1, L1.astype(np.uint16))
         put(w.L1f, l1_fragment_order(L1.astype(np.uint16)))
+        put(w.L1t, np.ascontiguousarray(L1.astype(np.uint16).T))
     return w, buf
 
 
@@ -75,7 +76,9 @@ def l1_fragment_order(L1):
     return out
 
 
-def _run_act(X, inv, L1, N=128):
+def _run_act(X, inv, L1, N=128, ws=False):
+    """Codes, scales and D of X from svdq_quantize_act (ws=False) or from the
+    forward's own activation kernel through svdq_quantize_act_ws (ws=True)."""
     M, K = X.shape
     r = 0 if L1 is None else L1.shape[1]
     w, buf = _weight_with(K, N, r, inv, L1)
@@ -84,8 +87,15 @@ def _run_act(X, inv, L1, N=128):
     codes = empty_u8(svdq.svdq_act_codes_bytes(M, K))
     scales = empty_u8(svdq.svdq_act_scales_bytes(M, K))
     D = t.empty((max(M, 1), max(r, 1)), dtype=t.int16, device="cuda")
-    svdq.svdq_quantize_act(Xd.data_ptr(), M, w, codes.data_ptr(), scales.data_ptr(),
-                           D.data_ptr() if r else 0, stream())
+    if ws:
+        nb = svdq.svdq_act_workspace_bytes(M, K, r)
+        wsb = empty_u8(nb)
+        with svdq.override(svdq.SVDQ_OVERRIDE_ACT_KERNEL, 2):
+            svdq.svdq_quantize_act_ws(Xd.data_ptr(), M, w, codes.data_ptr(), scales.data_ptr(),
+                                      D.data_ptr() if r else 0, wsb.data_ptr(), nb, stream())
+    else:
+        svdq.svdq_quantize_act(Xd.data_ptr(), M, w, codes.data_ptr(), scales.data_ptr(),
+                               D.data_ptr() if r else 0, stream())
     t.cuda.synchronize()
     nat = codes[: M * K // 2].cpu().numpy().reshape(M, K // 2)
     sn = scales[: svdq.svdq_act_scales_bytes(M, K)].cpu().numpy()
@@ -125,27 +135,33 @@ def _oracle_prep_from_export(W, lam, bias, exp, r):
 # S1: activation quantisation
 # ---------------------------------------------------------------------------
 
+KERNELS = pytest.mark.parametrize("ws", [False, True], ids=["act16", "act128"])
+
+
+@KERNELS
 @pytest.mark.parametrize("M,K,r", [(256, 512, 32), (1, 256, 16), (17, 768, 32), (129, 512, 64),
-                                   (300, 1024, 8), (64, 256, 0), (200, 512, 48)])
-def test_act_quant_parity(M, K, r):
-    _act_parity_case(M, K, r)
+                                   (300, 1024, 8), (64, 256, 0), (200, 512, 48), (1000, 3072, 32)])
+def test_act_quant_parity(M, K, r, ws):
+    _act_parity_case(M, K, r, ws)
 
 
+@KERNELS
 @pytest.mark.parametrize("ks", [1, 2, 3, 4, 6, 8])
 @pytest.mark.parametrize("r", [32, 64, 0])
-def test_act_quant_parity_k_split(ks, r):
-    """Clusters of ks CTAs sharing each 16-row block (the small-M path), each
-    CTA one of ks equal K ranges, partial D summed in the first CTA."""
+def test_act_quant_parity_k_split(ks, r, ws):
+    """K split forced to ks: clusters of ks CTAs sharing each 16-row block
+    (svdq_quantize_act), or ks CTAs per 128-row block whose float32 partials of
+    D the last one adds (the forward's kernel, through svdq_quantize_act_ws)."""
     with svdq.override(svdq.SVDQ_OVERRIDE_ACT_KSPLIT, ks):
-        _act_parity_case(40, 3072, r)
+        _act_parity_case(40 if not ws else 300, 3072, r, ws)
 
 
-def _act_parity_case(M, K, r):
+def _act_parity_case(M, K, r, ws=False):
     X, W, _, lam = _inputs(M, K, max(128, r), seed=M * 7 + K + r)
     inv = ref.inv_lambda_of(lam)
     rng = np.random.default_rng(5)
     L1 = gen.to_bf16_bits(rng.standard_normal((K, r)) * 0.3) if r else None
-    codes, scales, full, d = _run_act(X, inv, L1)
+    codes, scales, full, d = _run_act(X, inv, L1, ws=ws)
     o = ref.quantize_act(X, inv, L1)
     nbad = int((codes != o["x_codes"]).sum())
     assert nbad == 0, f"{nbad} code bytes differ"
@@ -155,7 +171,8 @@ def _act_parity_case(M, K, r):
         check_d(d, o["D"], o["D_abs"])
 
 
-def test_act_quant_rounding_cases():
+@KERNELS
+def test_act_quant_rounding_cases(ws):
     """Exact ties, scale ties, saturation, zero and negative-zero blocks (lambda = 1)."""
     K = 256
     ties = [6, 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5, -0.25, -0.75, -1.25, -1.75, -2.5, -3.5, -5, -0.0]
@@ -174,13 +191,14 @@ def test_act_quant_rounding_cases():
     rows.append(([6.0, 0.2501, 0.7499, 1.2501, 1.7499, 2.5001, 3.4999, 5.0001] * 2) * (K // 16))
     X = gen.to_bf16_bits(np.array(rows, dtype=np.float64))
     inv = np.ones(K, np.float32)
-    codes, scales, _, _ = _run_act(X, inv, None)
+    codes, scales, _, _ = _run_act(X, inv, _any_l1(K) if ws else None, ws=ws)
     o = ref.quantize_act(X, inv, None)
     assert np.array_equal(scales, o["x_scales"])
     assert np.array_equal(codes, o["x_codes"]), np.argwhere(codes != o["x_codes"])[:8]
 
 
-def test_act_quant_random_lambda_sweep():
+@KERNELS
+def test_act_quant_random_lambda_sweep(ws):
     """Many distinct float32 quotients: X and lambda random over wide ranges."""
     rng = np.random.default_rng(77)
     M, K = 512, 2048
@@ -188,10 +206,15 @@ def test_act_quant_random_lambda_sweep():
     X = gen.to_bf16_bits(x)
     lam = np.exp(rng.uniform(-3, 3, K)).astype(np.float32)
     inv = ref.inv_lambda_of(lam)
-    codes, scales, _, _ = _run_act(X, inv, None)
+    codes, scales, _, _ = _run_act(X, inv, _any_l1(K) if ws else None, ws=ws)
     o = ref.quantize_act(X, inv, None)
     assert np.array_equal(scales, o["x_scales"])
     assert int((codes != o["x_codes"]).sum()) == 0
+
+
+def _any_l1(K, r=16):
+    """Some L1 (codes and scales do not depend on it; the forward's kernel needs r > 0)."""
+    return gen.to_bf16_bits(np.random.default_rng(3).standard_normal((K, r)) * 0.3)
 
 
 # ---------------------------------------------------------------------------
@@ -305,6 +328,26 @@ def test_forward_parity(M, K, N, r, with_bias):
     o = ref.linear_forward(X, prep)
     yd = y_with_d(o["Y64"], o["D"], gpu_d(lin, dev_u16(X), M), exp["L2t"]) if r else None
     check_y(to_np_u16(Y.view(t.int16)), o["Y64"], "forward", y_given_gpu_d=yd)
+
+
+@pytest.mark.parametrize("M,K,N,r", [(256, 512, 512, 32), (129, 1024, 384, 16), (777, 3072, 1280, 64),
+                                     (3000, 1536, 256, 32), (1, 256, 256, 8)])
+def test_forward_parity_tensor_core_activation_kernel(M, K, N, r):
+    """The whole layer with the 128-row activation kernel forced (D on the tensor
+    cores, K split with float32 partials), at the strict bar."""
+    t = torch()
+    X, W, B, lam = _inputs(M, K, N, seed=13 * M + K + N + r)
+    lin, exp = _prepare(W, lam, B, r)
+    prep = _oracle_prep_from_export(W, lam, B, exp, r)
+    with svdq.override(svdq.SVDQ_OVERRIDE_ACT_KERNEL, 2):
+        Y = lin.forward(dev_u16(X).view(t.bfloat16))
+        t.cuda.synchronize()
+        Dg = gpu_d(lin, dev_u16(X), M)
+    o = ref.linear_forward(X, prep)
+    check_d(Dg, o["D"], o["D_abs"])
+    yd = y_with_d(o["Y64"], o["D"], Dg, exp["L2t"])
+    check_y(to_np_u16(Y.view(t.int16)), o["Y64"], "forward (128-row act)", y_given_gpu_d=yd)
+    assert svdq.svdq_get_device_status(stream()) == 0
 
 
 def test_forward_small_workload_end_to_end():

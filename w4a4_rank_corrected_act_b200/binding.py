@@ -39,7 +39,7 @@ class svdq_weight(ctypes.Structure):
         ("N", ctypes.c_int32), ("K", ctypes.c_int32), ("r", ctypes.c_int32),
         ("has_bias", ctypes.c_int32), ("format", ctypes.c_int32),
         ("w_codes", _P), ("w_scales", _P), ("L1", _P), ("L1f", _P), ("L2t", _P),
-        ("inv_lambda", _P), ("bias", _P),
+        ("inv_lambda", _P), ("bias", _P), ("L1t", _P),
     ]
 
 
@@ -58,6 +58,8 @@ SIGNATURES = {
     "svdq_weight_bind_format": (_I, [_P, _SZ, _I, _I, _I, _I, _I, _WP]),
     "svdq_prepare_weight": (_I, [_P, _P, _P, _WP, _P, _SZ, _P]),
     "svdq_quantize_act": (_I, [_P, _I, _WP, _P, _P, _P, _P]),
+    "svdq_act_workspace_bytes": (_SZ, [_I, _I, _I]),
+    "svdq_quantize_act_ws": (_I, [_P, _I, _WP, _P, _P, _P, _P, _SZ, _P]),
     "svdq_gemm": (_I, [_P, _P, _P, _I, _WP, _P, _P]),
     "svdq_linear_forward": (_I, [_P, _I, _WP, _P, _P, _SZ, _P]),
     "svdq_linear_forward_host": (_I, [_P, _I, _WP, _P, _P, _P, _P, _SZ, _P]),
@@ -176,6 +178,17 @@ def svdq_quantize_act(X: int, M: int, w: svdq_weight, x_codes: int, x_scales: in
     _call("svdq_quantize_act", X, M, ctypes.byref(w), x_codes, x_scales, D or None, stream or None)
 
 
+def svdq_act_workspace_bytes(M: int, K: int, r: int) -> int:
+    return int(lib().svdq_act_workspace_bytes(M, K, r))
+
+
+def svdq_quantize_act_ws(X: int, M: int, w: svdq_weight, x_codes: int, x_scales: int, D: int, ws: int,
+                         ws_bytes: int, stream: int) -> None:
+    """The forward's own activation kernel (128-row CTAs, D on the tensor cores)."""
+    _call("svdq_quantize_act_ws", X, M, ctypes.byref(w), x_codes, x_scales, D or None, ws, ws_bytes,
+          stream or None)
+
+
 def svdq_gemm(x_codes: int, x_scales: int, D: int, M: int, w: svdq_weight, Y: int,
               stream: int) -> None:
     _call("svdq_gemm", x_codes, x_scales, D or None, M, ctypes.byref(w), Y, stream or None)
@@ -269,6 +282,7 @@ SVDQ_OVERRIDE_ACT_KSPLIT = 1
 SVDQ_OVERRIDE_GEMM_BN = 2
 SVDQ_OVERRIDE_HOST_CHUNK_ROWS = 3
 SVDQ_OVERRIDE_SMALL_M = 4
+SVDQ_OVERRIDE_ACT_KERNEL = 5
 
 
 def svdq_set_override(which: int, value: int) -> None:

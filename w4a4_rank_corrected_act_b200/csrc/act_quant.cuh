@@ -303,4 +303,15 @@ __global__ void l1_fragment_kernel(const uint16_t* __restrict__ L1, int K, int r
   }
 }
 
+// L1 (K x r, row-major bf16) -> L1^T (r x K, row-major): the K-major operand
+// of the activation kernel's tensor-core product.
+__global__ void l1_transpose_kernel(const uint16_t* __restrict__ L1, int K, int r, uint16_t* __restrict__ L1t) {
+  const size_t total = static_cast<size_t>(K) * r;
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
+    const int j = static_cast<int>(i / K), k = static_cast<int>(i % K);
+    L1t[i] = L1[static_cast<size_t>(k) * r + j];
+  }
+}
+
 }  // namespace svdq

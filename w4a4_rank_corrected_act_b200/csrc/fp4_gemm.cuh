@@ -100,21 +100,6 @@ struct GemmCfg {
   static_assert(kSmemBytes <= 232448, "shared memory");
 };
 
-// Instruction descriptors (tcgen05.mma, 32-bit):
-//   kind::f16      : bits 4-5 D format (1 = f32), 7-9 A format (1 = bf16),
-//                    10-12 B format (1 = bf16), 15/16 A/B major (0 = K-major),
-//                    17-22 N >> 3, 24-28 M >> 4.
-//   kind::mxf4nvf4 : bits 4-5 B scale id, 7-9 A format (1 = E2M1), 10-12 B
-//                    format (1 = E2M1), 17-22 N >> 3, 23 scale type (0 = UE4M3),
-//                    24-28 M >> 4, 29-30 A scale id, 31 K size (0 = 64).
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
-         (static_cast<uint32_t>(M >> 4) << 24);
-}
-__host__ __device__ constexpr uint32_t idesc_nvfp4(int M, int N) {
-  return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
-         (static_cast<uint32_t>(M >> 4) << 24);
-}
 
 // Bias of columns n0 .. n0 + BN - 1, 16 bytes per lane (lane l holds columns
 // n0 + 8 l .. n0 + 8 l + 7); loaded before the accumulator is ready so that its

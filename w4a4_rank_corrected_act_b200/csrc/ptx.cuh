@@ -345,6 +345,22 @@ __device__ __forceinline__ void st_shared_cluster_f32(uint32_t cluster_addr, flo
 //   bits 49-51 base offset (0)         bit  52    LBO mode (0)
 //   bits 61-63 layout: 0 none, 2 128B swizzle, 4 64B swizzle, 6 32B swizzle
 // ---------------------------------------------------------------------------
+// Instruction descriptors (tcgen05.mma, 32-bit):
+//   kind::f16      : bits 4-5 D format (1 = f32), 7-9 A format (1 = bf16),
+//                    10-12 B format (1 = bf16), 15/16 A/B major (0 = K-major),
+//                    17-22 N >> 3, 24-28 M >> 4.
+//   kind::mxf4nvf4 : bits 4-5 B scale id, 7-9 A format (1 = E2M1), 10-12 B
+//                    format (1 = E2M1), 17-22 N >> 3, 23 scale type (0 = UE4M3),
+//                    24-28 M >> 4, 29-30 A scale id, 31 K size (0 = 64).
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+__host__ __device__ constexpr uint32_t idesc_nvfp4(int M, int N) {
+  return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
 enum : uint32_t { LAYOUT_NONE = 0, LAYOUT_SW128 = 2, LAYOUT_SW64 = 4, LAYOUT_SW32 = 6 };
 
 __device__ __forceinline__ uint64_t make_smem_desc(uint32_t saddr, uint32_t layout,

@@ -16,6 +16,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <random>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -27,6 +28,7 @@
 
 #include "svdq.h"
 #include "act_quant.cuh"
+#include "act128.cuh"
 #include "fp4_gemm.cuh"
 #include "int4.cuh"
 #include "prepare.cuh"
@@ -77,11 +79,11 @@ svdq_status check_weight(const svdq_weight* w) {
   if (s != SVDQ_OK) return s;
   if (w->w_codes == nullptr || w->w_scales == nullptr || w->inv_lambda == nullptr)
     return SVDQ_ERR_INVALID_ARG;
-  if (w->r > 0 && (w->L1 == nullptr || w->L1f == nullptr || w->L2t == nullptr))
+  if (w->r > 0 && (w->L1 == nullptr || w->L1f == nullptr || w->L2t == nullptr || w->L1t == nullptr))
     return SVDQ_ERR_INVALID_ARG;
   if (w->has_bias && w->bias == nullptr) return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(w->w_codes) || !aligned16(w->w_scales) || !aligned16(w->inv_lambda) ||
-      (w->r > 0 && (!aligned16(w->L1) || !aligned16(w->L1f) || !aligned16(w->L2t))) ||
+      (w->r > 0 && (!aligned16(w->L1) || !aligned16(w->L1f) || !aligned16(w->L2t) || !aligned16(w->L1t))) ||
       (w->has_bias && !aligned16(w->bias)))
     return SVDQ_ERR_MISALIGNED;
   return SVDQ_OK;
@@ -248,6 +250,64 @@ int act_k_split(int M, int K) {
   return ks;
 }
 
+// act128_kernel takes a layer when each CTA walks at least this many 64-column
+// stages (measured: at 6 stages, qkv at 1024x1024, the 16-row kernel is 4 us
+// faster; at 24, mlp_down and qkv at 18432 tokens, the tensor-core kernel is 6
+// and 14 us faster).
+constexpr int A128_MIN_STAGES = 12;
+
+// K split of act128_kernel: the largest ks <= A128_MAX_KS with K % (64 ks) == 0
+// and at most two CTAs per SM (128-row blocks x ks); SVDQ_OVERRIDE_ACT_KSPLIT
+// (svdq_set_override) replaces it when K % (64 ks) == 0.
+int a128_k_split(int M, int K) {
+  {
+    const int v = override_value(SVDQ_OVERRIDE_ACT_KSPLIT);
+    if (v >= 1 && v <= A128_MAX_KS && K % (64 * v) == 0) return v;
+  }
+  const int blocks = m_pad_of(M) / A128_ROWS;
+  int ks = 1;
+  for (int c = 2; c <= A128_MAX_KS; ++c)
+    if (K % (64 * c) == 0 && blocks * c <= 2 * num_sms()) ks = c;
+  return ks;
+}
+
+// A value no flag of an earlier call (nor, but with probability 2^-64, stale
+// workspace contents) holds: a per-process random key mixed with a counter.
+unsigned long long next_epoch() {
+  static const unsigned long long key = [] {
+    std::random_device rd;
+    return (static_cast<unsigned long long>(rd()) << 32) ^ rd() ^ 0x5DEECE66Dull;
+  }();
+  static std::atomic<unsigned long long> counter{0};
+  unsigned long long e = 0;
+  while (e == 0) e = key ^ ((counter.fetch_add(1) + 1) * 0x9E3779B97F4A7C15ull);
+  return e;
+}
+
+template <int R_PAD>
+svdq_status launch_act128(const CUtensorMap& tx, const CUtensorMap& tl1t, const A128Params& p, cudaStream_t st) {
+  constexpr uint32_t smem = A128Cfg<R_PAD>::kBytes;
+  {
+    const svdq_status so =
+        opt_in_smem(reinterpret_cast<const void*>(act128_kernel<R_PAD>), smem, "cudaFuncSetAttribute(act128)");
+    if (so != SVDQ_OK) return so;
+  }
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(p.M_pad / A128_ROWS * p.ks));
+  cfg.blockDim = dim3(A128_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, act128_kernel<R_PAD>, tx, tl1t, p);
+  if (e != cudaSuccess) return cuda_fail(e, "act128_kernel launch");
+  SVDQ_CHECK_LAUNCH("act128_kernel");
+  return SVDQ_OK;
+}
+
 template <int BN, int R_PAD, bool MLP = false>
 svdq_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
                         const CUtensorMap& tl2, const CUtensorMap& ty, const GemmParams& p,
@@ -391,9 +451,43 @@ svdq_status gemm_int4_impl(const uint8_t* x_codes, const uint8_t* x_scales, cons
 
 svdq_status quantize_act_impl(const uint16_t* X, int M, const svdq_weight* w, uint8_t* x_codes,
                               uint8_t* x_scales, uint16_t* D, cudaStream_t st, float* zero_ptr = nullptr,
-                              int zero_count = 0) {
+                              int zero_count = 0, float* dpart = nullptr, unsigned long long* flags = nullptr) {
   if (w->format == SVDQ_FORMAT_INT4) return quantize_act_int4_impl(X, M, w, x_codes, x_scales, D, st);
   const int K = w->K, r = w->r, rp = r_pad_of(r);
+  const int kernel_choice = override_value(SVDQ_OVERRIDE_ACT_KERNEL);
+  if (r > 0 && dpart != nullptr && flags != nullptr &&
+      (kernel_choice == 2 || (kernel_choice != 1 && K / (64 * a128_k_split(M, K)) >= A128_MIN_STAGES))) {
+    // 128-row CTAs, D on the tensor cores (needs the workspace for its K
+    // split), when every CTA has enough stages to amortise the split's
+    // cross-CTA reduction; the 16-row kernel otherwise
+    CUtensorMap tx{}, tl{};
+    svdq_status s = make_tmap(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, static_cast<uint64_t>(K) * 2, 64,
+                              A128_ROWS, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (s != SVDQ_OK) return s;
+    s = make_tmap(&tl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->L1t, K, r, static_cast<uint64_t>(K) * 2, 64, rp,
+                  CU_TENSOR_MAP_SWIZZLE_128B);
+    if (s != SVDQ_OK) return s;
+    A128Params p{};
+    p.inv_lambda = w->inv_lambda;
+    p.x_codes = x_codes;
+    p.x_scales = x_scales;
+    p.D = D;
+    p.dpart = dpart;
+    p.flags = flags;
+    p.epoch = next_epoch();
+    p.M = M;
+    p.K = K;
+    p.r = r;
+    p.M_pad = m_pad_of(M);
+    p.ks = a128_k_split(M, K);
+    p.zero_ptr = zero_ptr;
+    p.zero_count = zero_count;
+    switch (rp) {
+      case 16: return launch_act128<16>(tx, tl, p, st);
+      case 32: return launch_act128<32>(tx, tl, p, st);
+      default: return launch_act128<64>(tx, tl, p, st);
+    }
+  }
   CUtensorMap tx{};
   svdq_status s = make_tmap(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M,
                             static_cast<uint64_t>(K) * 2, ACT_SUB, ACT_ROWS,
@@ -576,18 +670,38 @@ struct ActWs {
   uint8_t* codes;
   uint8_t* scales;
   uint16_t* D;
+  float* dpart;                 // act128_kernel's K-split partials of D (r > 0)
+  unsigned long long* flags;    // and their flags
 };
+
+// Bytes of the K-split partials of D ([M_pad / 128][A128_MAX_KS][r][128]
+// float32) and of their flags ([M_pad / 128][A128_MAX_KS]), each 256-aligned;
+// 0 for r = 0.
+size_t act_partials_bytes(int M, int r, size_t* flags_off) {
+  if (r == 0) {
+    if (flags_off) *flags_off = 0;
+    return 0;
+  }
+  const size_t part = align_up(static_cast<size_t>(A128_MAX_KS) * m_pad_of(M) * r * 4, kAlign);
+  const size_t fl = align_up(static_cast<size_t>(m_pad_of(M) / A128_ROWS) * A128_MAX_KS * 8, kAlign);
+  if (flags_off) *flags_off = part;
+  return part + fl;
+}
 
 size_t act_ws_layout(int M, int K, int r, uint8_t* base, ActWs* out) {
   const size_t c = align_up(static_cast<size_t>(M) * (K / 2), kAlign);
   const size_t s = align_up(static_cast<size_t>(m_pad_of(M)) * (K / 16), kAlign);
   const size_t d = align_up(static_cast<size_t>(M) * r * 2, kAlign);
+  size_t flags_off = 0;
+  const size_t pb = act_partials_bytes(M, r, &flags_off);
   if (out != nullptr) {
     out->codes = base;
     out->scales = base + c;
     out->D = r > 0 ? reinterpret_cast<uint16_t*>(base + c + s) : nullptr;
+    out->dpart = r > 0 ? reinterpret_cast<float*>(base + c + s + d) : nullptr;
+    out->flags = r > 0 ? reinterpret_cast<unsigned long long*>(base + c + s + d + flags_off) : nullptr;
   }
-  return c + s + d;
+  return c + s + d + pb;
 }
 
 // Workspace of the few-token path (M <= 32): activation codes M x K/2, the
@@ -640,6 +754,7 @@ size_t weight_layout(int N, int K, int r, int has_bias, uint8_t* base, svdq_weig
   uint8_t* l2t = take(static_cast<size_t>(N) * r * 2);
   uint8_t* inv = take(static_cast<size_t>(K) * 4);
   uint8_t* bias = has_bias ? take(static_cast<size_t>(N) * 2) : nullptr;
+  uint8_t* l1t = take(static_cast<size_t>(K) * r * 2);
   if (out != nullptr) {
     out->N = N;
     out->K = K;
@@ -653,6 +768,7 @@ size_t weight_layout(int N, int K, int r, int has_bias, uint8_t* base, svdq_weig
     out->L2t = r > 0 ? reinterpret_cast<uint16_t*>(l2t) : nullptr;
     out->inv_lambda = reinterpret_cast<float*>(inv);
     out->bias = reinterpret_cast<uint16_t*>(bias);
+    out->L1t = r > 0 ? reinterpret_cast<uint16_t*>(l1t) : nullptr;
   }
   return off;
 }
@@ -714,7 +830,7 @@ svdq_status forward_impl(const uint16_t* X, int M, const svdq_weight* w, uint16_
   if (small_m_path(M, w)) return small_forward_impl(X, M, w, Y, ws, st, head_dim);
   ActWs a;
   act_ws_layout(M, w->K, w->r, static_cast<uint8_t*>(ws), &a);
-  svdq_status s = quantize_act_impl(X, M, w, a.codes, a.scales, a.D, st);
+  svdq_status s = quantize_act_impl(X, M, w, a.codes, a.scales, a.D, st, nullptr, 0, a.dpart, a.flags);
   if (s != SVDQ_OK) return s;
   return gemm_impl(a.codes, a.scales, a.D, M, w, Y, st, head_dim);
 }
@@ -745,7 +861,8 @@ svdq_status mlp_forward_impl(const uint16_t* X, int M, const svdq_weight* up, co
   mlp_ws_layout(M, up->K, up->N, up->r, down->r, static_cast<uint8_t*>(ws), &m);
   const int nd = M * down->r;
   // the up-projection's activation kernel, which also clears the D accumulator
-  svdq_status s = quantize_act_impl(X, M, up, m.up.codes, m.up.scales, m.up.D, st, m.d_acc, nd);
+  svdq_status s = quantize_act_impl(X, M, up, m.up.codes, m.up.scales, m.up.D, st, m.d_acc, nd, m.up.dpart,
+                                    m.up.flags);
   if (s != SVDQ_OK) return s;
   GemmParams e{};
   e.inv_lambda_next = down->inv_lambda;
@@ -1145,6 +1262,7 @@ svdq_status svdq_prepare_weight(const uint16_t* W, const float* lambda, const ui
     prep_sign_kernel<<<r, 256, 0, st>>>(pw.L1f, pw.L2f, N, K, r);
     prep_round_kernel<<<nsm * 4, 256, 0, st>>>(pw.L1f, pw.L2f, N, K, r, w->L1, w->L2t);
     l1_fragment_kernel<<<nsm * 2, 256, 0, st>>>(w->L1, K, r, w->L1f);
+    l1_transpose_kernel<<<nsm * 2, 256, 0, st>>>(w->L1, K, r, w->L1t);
     e = cudaGetLastError();
     if (e != cudaSuccess) return fail(cuda_fail(e, "prepare factor kernels"));
   }
@@ -1179,6 +1297,31 @@ svdq_status svdq_quantize_act(const uint16_t* X, int M, const svdq_weight* w, ui
   if (!aligned16(X) || !aligned16(x_codes) || !aligned16(x_scales) || (w->r > 0 && !aligned16(D)))
     return SVDQ_ERR_MISALIGNED;
   return quantize_act_impl(X, M, w, x_codes, x_scales, D, static_cast<cudaStream_t>(stream));
+}
+
+size_t svdq_act_workspace_bytes(int M, int K, int r) {
+  if (M < 0 || check_layer_shape(128, K, r) != SVDQ_OK) return 0;
+  return std::max<size_t>(act_partials_bytes(M, r, nullptr), kAlign);
+}
+
+svdq_status svdq_quantize_act_ws(const uint16_t* X, int M, const svdq_weight* w, uint8_t* x_codes,
+                                 uint8_t* x_scales, uint16_t* D, void* ws, size_t ws_bytes, void* stream) {
+  svdq_status s = check_weight(w);
+  if (s != SVDQ_OK) return s;
+  if (M < 0) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  if (X == nullptr || x_codes == nullptr || x_scales == nullptr || (w->r > 0 && D == nullptr) || ws == nullptr)
+    return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(x_codes) || !aligned16(x_scales) || (w->r > 0 && !aligned16(D)) ||
+      !aligned16(ws))
+    return SVDQ_ERR_MISALIGNED;
+  if (ws_bytes < act_partials_bytes(M, w->r, nullptr)) return SVDQ_ERR_WORKSPACE_TOO_SMALL;
+  size_t flags_off = 0;
+  act_partials_bytes(M, w->r, &flags_off);
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  return quantize_act_impl(X, M, w, x_codes, x_scales, D, static_cast<cudaStream_t>(stream), nullptr, 0,
+                           w->r > 0 ? reinterpret_cast<float*>(b) : nullptr,
+                           w->r > 0 ? reinterpret_cast<unsigned long long*>(b + flags_off) : nullptr);
 }
 
 svdq_status svdq_gemm(const uint8_t* x_codes, const uint8_t* x_scales, const uint16_t* D, int M,
@@ -1412,6 +1555,8 @@ svdq_status svdq_weight_import(const svdq_weight* w, const uint8_t* host_codes, 
     SVDQ_CUDA(cudaMemcpyAsync(w->L2t, host_L2t, N * r * 2, cudaMemcpyHostToDevice, st));
     l1_fragment_kernel<<<num_sms() * 2, 256, 0, st>>>(w->L1, w->K, w->r, w->L1f);
     SVDQ_CHECK_LAUNCH("l1_fragment_kernel");
+    l1_transpose_kernel<<<num_sms() * 2, 256, 0, st>>>(w->L1, w->K, w->r, w->L1t);
+    SVDQ_CHECK_LAUNCH("l1_transpose_kernel");
   }
   SVDQ_CUDA(cudaMemcpyAsync(w->inv_lambda, host_inv_lambda, K * 4, cudaMemcpyHostToDevice, st));
   if (host_bias) SVDQ_CUDA(cudaMemcpyAsync(w->bias, host_bias, N * 2, cudaMemcpyHostToDevice, st));
