@@ -190,6 +190,20 @@ def _run_for(seconds, flush, step):
             step()
         torch.cuda.synchronize()
 
+def act_kernel_name(M, K, r, int4, sms=148):
+    """The activation kernel the forward runs (the library's routing rule): the
+    tensor-core one when r > 0 and each of its 128-row CTAs, K split up to 8
+    ways at two CTAs per SM, walks at least 12 stages of 64 columns."""
+    if int4:
+        return "act_quant_int4_kernel"
+    blocks = (M + 127) // 128
+    ks = 1
+    for c in range(2, 9):
+        if K % (64 * c) == 0 and blocks * c <= 2 * sms:
+            ks = c
+    return "act128_kernel" if r > 0 and K // (64 * ks) >= 12 else "act_quant_kernel"
+
+
 def kernel_rooflines(M, N, K, r, gemm_ms, act_ms, int4, workload):
     """Roofline entries of the GEMM (the dominant kernel) and the activation
     kernel from their event-timed launch durations (ms): algorithmic bytes or
@@ -239,7 +253,7 @@ def kernel_rooflines(M, N, K, r, gemm_ms, act_ms, int4, workload):
         "arithmetic_intensity_flop_per_byte": round(flops / gemm_bytes, 1),
         "launch_us": round(gemm_ms * 1e3, 2),
     })
-    act = {"kernel": "act_quant_int4_kernel" if int4 else "act_quant_kernel", "bound": "hbm",
+    act = {"kernel": act_kernel_name(M, K, r, int4), "bound": "hbm",
            "achieved": round(act_gbs, 1),
            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(act_gbs / peaks["hbm_gbs"], 4),
            "algorithmic_bytes_per_launch": act_bytes, "launch_us": round(act_ms * 1e3, 2),
@@ -457,7 +471,30 @@ def measure_mlp_pair(steps, warmup, st, flush):
            "tflops": round(flops / (us * 1e-6) / 1e12, 1),
            "us_isolated_p50": round(float(np.percentile(iso, 50)) * 1e3, 2), "graph": graph,
            "kernels_per_pair": 4 if sd.r else 3}
-    del up, down, copies
+    del copies
+    # The same pair unfused, for comparison: the two layers through
+    # svdq_linear_forward with H = GELU-tanh(Y_up) in bf16 between them (that
+    # one elementwise pass is PyTorch's, not this library's: a comparison leg).
+    nbu, nbd = up.workspace_bytes(M), down.workspace_bytes(M)
+    ucopies = []
+    for i in range(2):
+        ucopies.append((X if i == 0 else X.clone(), torch.empty((M, F), dtype=torch.bfloat16, device="cuda"),
+                        torch.empty((M, N), dtype=torch.int16, device="cuda"),
+                        torch.empty(nbu, dtype=torch.uint8, device="cuda"),
+                        torch.empty(nbd, dtype=torch.uint8, device="cuda")))
+
+    def ustep(i):
+        Xi, Hi, Yi, wu, wd = ucopies[i % len(ucopies)]
+        svdq.svdq_linear_forward(Xi.data_ptr(), M, up.w, Hi.data_ptr(), wu.data_ptr(), nbu, sh)
+        torch.ops.aten.gelu_(Hi, approximate="tanh")
+        svdq.svdq_linear_forward(Hi.data_ptr(), M, down.w, Yi.data_ptr(), wd.data_ptr(), nbd, sh)
+
+    utotal, _ = time_back_to_back(ustep, steps, warmup, st)
+    uus = utotal / steps * 1e3
+    out["unfused_with_gelu"] = {"us_per_pair": round(uus, 2), "tflops": round(flops / (uus * 1e-6) / 1e12, 1),
+                                "note": "svdq_linear_forward (up), PyTorch GELU-tanh in bf16, "
+                                        "svdq_linear_forward (down)"}
+    del up, down, ucopies
     torch.cuda.empty_cache()
     return out
 
@@ -578,7 +615,13 @@ def run_native(args):
 
     # dominant kernel alone: the FP4 GEMM (svdq_gemm on the act kernel's output),
     # and the activation kernel alone, each timed with events on this stream
-    a = svdq.svdq_quantize_act
+    # the forward's own activation kernel (svdq_quantize_act_ws: the 16-row
+    # kernel or, with enough K per CTA, the one with D on the tensor cores)
+    nba = svdq.svdq_act_workspace_bytes(M, K, r)
+    aws = torch.empty(nba, dtype=torch.uint8, device="cuda")
+
+    def a(Xp, Mm, w, cp, sp, dp, s_):
+        svdq.svdq_quantize_act_ws(Xp, Mm, w, cp, sp, dp, aws.data_ptr(), nba, s_)
     codes_t = torch.empty(svdq.svdq_act_codes_bytes(M, K), dtype=torch.uint8, device="cuda")
     scales_t = torch.empty(svdq.svdq_act_scales_bytes(M, K), dtype=torch.uint8, device="cuda")
     d_t = torch.empty((M, max(r, 1)), dtype=torch.int16, device="cuda")
