@@ -564,9 +564,12 @@ __global__ void __launch_bounds__(MLP ? GEMM_MLP_THREADS : GEMM_THREADS, 1)
       const uint32_t tx_lr = (GEMM_BM + BN) * R_PAD * 2;
       // Programmatic dependent launch: this grid may start while the kernel
       // that writes the activation codes, scales and D is still running.  The
-      // weight halves of the first S stages are loaded at once; their
-      // activation halves wait for that kernel (griddepcontrol.wait), as does
-      // everything after them.  The stage barriers count both halves' bytes.
+      // weight half of the first stage is loaded at once; its activation half
+      // waits for that kernel (griddepcontrol.wait), as does everything after
+      // it.  (Deeper early weight loads compete with that kernel's own reads
+      // of X: with the first four stages early the qkv layer took 0.5 us
+      // longer back to back.)  The stage barriers count both halves' bytes.
+      constexpr int kEarlyStages = 1;
       struct Deferred {
         int stage, kb, m0, mb;   // kb < 0: the low-rank slot (D tile)
       };
@@ -595,7 +598,7 @@ __global__ void __launch_bounds__(MLP ? GEMM_MLP_THREADS : GEMM_THREADS, 1)
           load_activation(q);
         } else {
           deferred[ndeferred++] = q;
-          if (ndeferred == S) meet_dependency();   // the ring is full: nothing more to overlap
+          if (ndeferred == kEarlyStages) meet_dependency();
         }
       };
       bool ok = true;
