@@ -29,9 +29,16 @@ def _to_heads(Y, head_dim):
 
 # (M, K, N, r, head_dim): ragged M, r = 0 / 16 / 32, and one shape with more
 # tiles than SMs so that CTAs store tiles through both epilogue paths
+@pytest.mark.parametrize("act_kernel", [0, 2], ids=["auto", "act128"])
 @pytest.mark.parametrize("M,K,N,r,hd", [(300, 512, 768, 32, 128), (129, 1024, 512, 16, 64),
                                          (40, 768, 384, 0, 32), (2048, 256, 2048, 32, 128)])
-def test_heads_layout_matches_row_major(M, K, N, r, hd):
+def test_heads_layout_matches_row_major(M, K, N, r, hd, act_kernel):
+    """act_kernel 2 forces the 128-row activation kernel (D on the tensor cores)."""
+    with svdq.override(svdq.SVDQ_OVERRIDE_ACT_KERNEL, act_kernel):
+        _heads_case(M, K, N, r, hd)
+
+
+def _heads_case(M, K, N, r, hd):
     t = torch()
     lin, d = _layer(M, K, N, r, seed=M + K + N + hd)
     X = dev_u16(d["X"])

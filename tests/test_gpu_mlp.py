@@ -124,6 +124,14 @@ def test_mlp_pair_parity(M, K, F, N, r_up, r_down, bias):
     _check(X, M, up, down, Y_up, H_ref, b2, f"mlp {M}x{K}x{F}x{N}")
 
 
+def test_mlp_pair_parity_tensor_core_activation_kernel():
+    """The pair with the up-projection's activation kernel forced to the 128-row
+    kernel (D on the tensor cores, K split with float32 partials)."""
+    with svdq.override(svdq.SVDQ_OVERRIDE_ACT_KERNEL, 2):
+        X, up, down, Y_up, H_ref, b2 = _pair(300, 1536, 1024, 512, 32, 32, seed=31, bias=True)
+        _check(X, 300, up, down, Y_up, H_ref, b2, "mlp (128-row activation kernel)")
+
+
 def test_mlp_pair_matches_the_unfused_pair():
     """The fused pair against the same two layers run one after the other
     (svdq_linear_forward, GELU of the bf16 output in float64, svdq_linear_forward)."""
