@@ -183,23 +183,27 @@ __global__ void __launch_bounds__(A128_THREADS, 2)
     }
   } else {
     // ------------------------------------------------------- quantiser warps
-    const int chunk16 = lane & 7, rsub = lane >> 3;
+    // Lane l quantises the 16-column block l % 4 of rows l / 4 and l / 4 + 8 of
+    // the warp's 16: a whole block per thread, so no lane pair exchanges its
+    // maximum.  The block's two 16-byte chunks sit at toff and toff ^ 16 (the
+    // 128-byte swizzle keeps them in the same row, next to each other).
+    const int blk = lane & 3, rsub = lane >> 2;
     const uint32_t half_k = static_cast<uint32_t>(p.K) >> 1;
-    uint32_t toff[4];
-    uint8_t* cptr[4];
-    uint8_t* sptr[4];
+    uint32_t toff[2];
+    uint8_t* cptr[2];
+    uint8_t* sptr[2];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int row = warp * 16 + i * 4 + rsub, grow = row0 + row;
-      toff[i] = swz(static_cast<uint32_t>(row * 128 + chunk16 * 16), 3);
-      cptr[i] = grow < p.M ? p.x_codes + static_cast<size_t>(grow) * half_k + 4 * chunk16 : nullptr;
-      sptr[i] = p.x_scales + sf_offset(static_cast<uint32_t>(grow), 0, static_cast<uint32_t>(p.K)) + chunk16 / 2;
+    for (int i = 0; i < 2; ++i) {
+      const int row = warp * 16 + i * 8 + rsub, grow = row0 + row;
+      toff[i] = swz(static_cast<uint32_t>(row * 128 + blk * 32), 3);
+      cptr[i] = grow < p.M ? p.x_codes + static_cast<size_t>(grow) * half_k + 8 * blk : nullptr;
+      sptr[i] = p.x_scales + sf_offset(static_cast<uint32_t>(grow), 0, static_cast<uint32_t>(p.K)) + blk;
     }
-    float4 ni0, ni1;
+    float4 ni[4];
     auto load_inv = [&](int j) {
-      const float* src = p.inv_lambda + (sub0 + j) * 64 + 8 * chunk16;
-      ni0 = __ldg(reinterpret_cast<const float4*>(src));
-      ni1 = __ldg(reinterpret_cast<const float4*>(src + 4));
+      const float4* src = reinterpret_cast<const float4*>(p.inv_lambda + (sub0 + j) * 64 + 16 * blk);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) ni[u] = __ldg(src + u);
     };
     if (nsub > 0) load_inv(0);
     const float y6 = tab[0x4C].y;   // E4M3 code 0x4C is 6.0: RN(1/6)
@@ -207,34 +211,40 @@ __global__ void __launch_bounds__(A128_THREADS, 2)
     for (int j = 0; j < nsub; ++j) {
       const int s = j % S;
       const int col0 = (sub0 + j) * 64;
-      const uint64_t ninv2[4] = {f32x2_pack(-ni0.x, -ni0.y), f32x2_pack(-ni0.z, -ni0.w),
-                                 f32x2_pack(-ni1.x, -ni1.y), f32x2_pack(-ni1.z, -ni1.w)};
+      uint64_t ninv2[8];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        ninv2[2 * u] = f32x2_pack(-ni[u].x, -ni[u].y);
+        ninv2[2 * u + 1] = f32x2_pack(-ni[u].z, -ni[u].w);
+      }
       if (j + 1 < nsub) load_inv(j + 1);
       if (!mbar_wait(full_bar(s), static_cast<uint32_t>(j / S) & 1u, abort_flag, KID_ACT128, 3)) break;
       uint8_t* tile = smem + static_cast<uint32_t>(s) * Cfg::kStage;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint4 raw = *reinterpret_cast<const uint4*>(tile + toff[i]);
-        const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+      for (int i = 0; i < 2; ++i) {
+        const uint4 r0 = *reinterpret_cast<const uint4*>(tile + toff[i]);
+        const uint4 r1 = *reinterpret_cast<const uint4*>(tile + (toff[i] ^ 16u));
+        const uint32_t w8[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
         // -Xhat = f32(x * (-1/lambda)), element 2u in the low half of pair u
-        uint64_t nxh[4];
+        uint64_t nxh[8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-          nxh[u] = f32x2_mul(f32x2_pack(__uint_as_float(w4[u] << 16), __uint_as_float(w4[u] & 0xFFFF0000u)),
+        for (int u = 0; u < 8; ++u)
+          nxh[u] = f32x2_mul(f32x2_pack(__uint_as_float(w8[u] << 16), __uint_as_float(w8[u] & 0xFFFF0000u)),
                              ninv2[u]);
         uint32_t sc;
-        const uint32_t codes = nvfp4_quant_half_block_x2(nxh, tab, six, neg_y6, sc);
-        if (cptr[i] != nullptr) *reinterpret_cast<uint32_t*>(cptr[i] + (col0 >> 1)) = codes;
-        if ((chunk16 & 1) == 0) sptr[i][static_cast<size_t>(col0 >> 6) * 512] = static_cast<uint8_t>(sc);
+        const uint64_t codes = nvfp4_quant_block16_x2(nxh, tab, six, neg_y6, sc);
+        if (cptr[i] != nullptr) *reinterpret_cast<uint64_t*>(cptr[i] + (col0 >> 1)) = codes;
+        sptr[i][static_cast<size_t>(col0 >> 6) * 512] = static_cast<uint8_t>(sc);
         // bf16(-Xhat) = -bf16(Xhat) in place: the MMA's A operand (negated back at the end)
-        uint32_t o[4];
+        uint32_t o[8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < 8; ++u) {
           float lo, hi;
           f32x2_unpack(nxh[u], lo, hi);
           o[u] = pack_bf16x2(lo, hi);
         }
         *reinterpret_cast<uint4*>(tile + toff[i]) = make_uint4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<uint4*>(tile + (toff[i] ^ 16u)) = make_uint4(o[4], o[5], o[6], o[7]);
       }
       // the generic-proxy writes of the tile before the tensor core reads it
       fence_proxy_async_smem();

@@ -17,8 +17,8 @@
 // first CTA's shared memory.  Each warp
 // streams its sub-tiles through a private 4-slot TMA ring (16 x 64 bf16 boxes,
 // 128-byte swizzle), so no block-wide synchronisation happens until the final
-// reduction of D.  In a slot, lane pairs quantise 16-element blocks in
-// registers and write bf16(Xhat) back in place; ldmatrix then feeds
+// reduction of D.  In a slot, each lane quantises two whole 16-element blocks
+// in registers and writes bf16(Xhat) back in place; ldmatrix then feeds
 // mma.sync m16n8k16 with that tile, the B fragments of L1 coming straight from
 // L2 in the fragment order the weight stores them in.  X crosses HBM once.
 #pragma once
@@ -138,30 +138,23 @@ __global__ void __launch_bounds__(ACT_THREADS, R_PAD > 32 ? 1 : 2)
 #pragma unroll
     for (int i = 0; i < 4; ++i) acc[t][i] = 0.0f;
   const uint32_t half_k = static_cast<uint32_t>(p.K) >> 1;
-  const int chunk16 = lane & 7, rsub = lane >> 3;
-  // 1/lambda of this lane's 8 columns, one sub-tile ahead
-  float4 ni0 = make_float4(0.f, 0.f, 0.f, 0.f), ni1 = ni0;
-  auto load_inv = [&](int j) {
-    const float* src = p.inv_lambda + (sub0 + warp + ACT_WARPS * j) * ACT_SUB + 8 * chunk16;
-    ni0 = __ldg(reinterpret_cast<const float4*>(src));
-    ni1 = __ldg(reinterpret_cast<const float4*>(src + 4));
-  };
-  if (my_count > 0) load_inv(0);
+  // lane l quantises the 16-column block l % 4 of rows l / 4 and l / 4 + 8: a
+  // whole block per thread, so no lane pair exchanges its maximum
+  const int blk = lane & 3, rsub = lane >> 2;
   const float y6 = tab[0x4C].y;   // E4M3 code 0x4C is 6.0: RN(1/6)
   const uint64_t six = f32x2_pack(6.0f, 6.0f), neg_y6 = f32x2_pack(-y6, -y6);
-  // row-dependent addresses, fixed for the whole K range: the 16 bytes of
-  // row 4 i + l / 8 in a (swizzled) sub-tile, its codes (null past M) and its
-  // scale bytes of column group 0 (one byte per 16-element block, written by
-  // the lower lane of each pair)
-  uint32_t toff[ACT_ROWS / 4];
-  uint8_t* cptr[ACT_ROWS / 4];
-  uint8_t* sptr[ACT_ROWS / 4];
+  // row-dependent addresses, fixed for the whole K range: the block's first
+  // 16 bytes in row 8 i + l / 4 of a (swizzled) sub-tile (the second 16 sit at
+  // toff ^ 16), its codes (null past M) and its scale byte of column group 0
+  uint32_t toff[ACT_ROWS / 8];
+  uint8_t* cptr[ACT_ROWS / 8];
+  uint8_t* sptr[ACT_ROWS / 8];
 #pragma unroll
-  for (int i = 0; i < ACT_ROWS / 4; ++i) {
-    const int row = i * 4 + rsub, grow = row0 + row;
-    toff[i] = swz(static_cast<uint32_t>(row * 128 + chunk16 * 16), 3);
-    cptr[i] = grow < p.M ? p.x_codes + static_cast<size_t>(grow) * half_k + 4 * chunk16 : nullptr;
-    sptr[i] = p.x_scales + sf_offset(static_cast<uint32_t>(grow), 0, static_cast<uint32_t>(p.K)) + chunk16 / 2;
+  for (int i = 0; i < ACT_ROWS / 8; ++i) {
+    const int row = i * 8 + rsub, grow = row0 + row;
+    toff[i] = swz(static_cast<uint32_t>(row * 128 + blk * 32), 3);
+    cptr[i] = grow < p.M ? p.x_codes + static_cast<size_t>(grow) * half_k + 8 * blk : nullptr;
+    sptr[i] = p.x_scales + sf_offset(static_cast<uint32_t>(grow), 0, static_cast<uint32_t>(p.K)) + blk;
   }
   int jj = 0;
   for (; jj < my_count; ++jj) {
@@ -178,40 +171,54 @@ __global__ void __launch_bounds__(ACT_THREADS, R_PAD > 32 ? 1 : 2)
           if (t < nt_count)
             bfr[ks][t] = __ldg(f + ((static_cast<size_t>(col0 / 16 + ks) * nt_count + t) * 32 + lane));
     }
-    // -1/lambda: the quantiser takes -Xhat (see nvfp4_quant_half_block_x2)
-    const uint64_t ninv2[4] = {f32x2_pack(-ni0.x, -ni0.y), f32x2_pack(-ni0.z, -ni0.w),
-                               f32x2_pack(-ni1.x, -ni1.y), f32x2_pack(-ni1.z, -ni1.w)};
-    if (jj + 1 < my_count) load_inv(jj + 1);
+    // 1/lambda of this lane's 16 columns (L1-resident after the first sub-tiles),
+    // in flight while the tile lands; loaded per sub-tile rather than one ahead,
+    // which would hold 16 more registers across the loop
+    float4 ni[4];
+    {
+      const float4* src = reinterpret_cast<const float4*>(p.inv_lambda + col0 + 16 * blk);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) ni[u] = __ldg(src + u);
+    }
     if (!mbar_wait(bar(slot), (jj / ACT_RING) & 1, abort_flag, KID_ACT, 1)) break;
+    // -1/lambda: the quantiser takes -Xhat (see nvfp4_quant_block16_x2)
+    uint64_t ninv2[8];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      ninv2[2 * u] = f32x2_pack(-ni[u].x, -ni[u].y);
+      ninv2[2 * u + 1] = f32x2_pack(-ni[u].z, -ni[u].w);
+    }
     uint8_t* tile = smem + (ring - smem_u32(smem)) + slot * ACT_SUB_BYTES;
 
 #pragma unroll
-    for (int i = 0; i < ACT_ROWS / 4; ++i) {
+    for (int i = 0; i < ACT_ROWS / 8; ++i) {
       const uint32_t off = toff[i];
-      const uint4 raw = *reinterpret_cast<const uint4*>(tile + off);
-      const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+      const uint4 r0 = *reinterpret_cast<const uint4*>(tile + off);
+      const uint4 r1 = *reinterpret_cast<const uint4*>(tile + (off ^ 16u));
+      const uint32_t w8[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
       // -Xhat = f32(x * (-1/lambda)) (exactly the negated product), element 2u
       // in the low half of pair u
-      uint64_t nxh[4];
+      uint64_t nxh[8];
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-        nxh[u] = f32x2_mul(f32x2_pack(__uint_as_float(w4[u] << 16), __uint_as_float(w4[u] & 0xFFFF0000u)),
+      for (int u = 0; u < 8; ++u)
+        nxh[u] = f32x2_mul(f32x2_pack(__uint_as_float(w8[u] << 16), __uint_as_float(w8[u] & 0xFFFF0000u)),
                            ninv2[u]);
       uint32_t sc;
-      const uint32_t codes = nvfp4_quant_half_block_x2(nxh, tab, six, neg_y6, sc);
-      if (cptr[i] != nullptr) *reinterpret_cast<uint32_t*>(cptr[i] + (col0 >> 1)) = codes;
-      if ((chunk16 & 1) == 0) sptr[i][static_cast<size_t>(col0 >> 6) * 512] = static_cast<uint8_t>(sc);
+      const uint64_t codes = nvfp4_quant_block16_x2(nxh, tab, six, neg_y6, sc);
+      if (cptr[i] != nullptr) *reinterpret_cast<uint64_t*>(cptr[i] + (col0 >> 1)) = codes;
+      sptr[i][static_cast<size_t>(col0 >> 6) * 512] = static_cast<uint8_t>(sc);
       if (R_PAD > 0) {
         // bf16(-Xhat) = -bf16(Xhat): the tile holds the negated operand, and the
         // product with L1 is negated back when D is written
-        uint32_t o[4];
+        uint32_t o[8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < 8; ++u) {
           float lo, hi;
           f32x2_unpack(nxh[u], lo, hi);
           o[u] = pack_bf16x2(lo, hi);
         }
         *reinterpret_cast<uint4*>(tile + off) = make_uint4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<uint4*>(tile + (off ^ 16u)) = make_uint4(o[4], o[5], o[6], o[7]);
       }
     }
 
