@@ -51,6 +51,7 @@ _CSRC = os.path.join(ROOT, "w4a4_rank_corrected_act_b200", "csrc")
 GEMM_SRC = [os.path.join(_CSRC, f) for f in ("fp4_gemm.cuh", "ptx.cuh", "nvfp4.cuh")]
 ACT_SRC = [os.path.join(_CSRC, f) for f in ("act_quant.cuh", "ptx.cuh", "nvfp4.cuh")]
 INT4_SRC = [os.path.join(_CSRC, f) for f in ("int4.cuh", "act_quant.cuh", "ptx.cuh", "nvfp4.cuh")]
+A128_SRC = [os.path.join(_CSRC, f) for f in ("act128.cuh", "ptx.cuh", "nvfp4.cuh")]
 I8_OVER_BF16 = 2.0                # nominal dense ratio int8 : bf16 (4.5 / 2.25 POPS)
 
 
@@ -253,12 +254,18 @@ def kernel_rooflines(M, N, K, r, gemm_ms, act_ms, int4, workload):
         "arithmetic_intensity_flop_per_byte": round(flops / gemm_bytes, 1),
         "launch_us": round(gemm_ms * 1e3, 2),
     })
-    act = {"kernel": act_kernel_name(M, K, r, int4), "bound": "hbm",
+    act_kernel = act_kernel_name(M, K, r, int4)
+    if int4:
+        act_traffic = _profile_traffic(INT4_SRC, f"act_quant_int4_{workload}.txt")
+    elif act_kernel == "act128_kernel":
+        act_traffic = _profile_traffic(A128_SRC, f"act128_{workload}.txt")
+    else:
+        act_traffic = _profile_traffic(ACT_SRC, f"act_quant_{workload}.txt")
+    act = {"kernel": act_kernel, "bound": "hbm",
            "achieved": round(act_gbs, 1),
            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(act_gbs / peaks["hbm_gbs"], 4),
            "algorithmic_bytes_per_launch": act_bytes, "launch_us": round(act_ms * 1e3, 2),
-           "traffic": (_profile_traffic(INT4_SRC, f"act_quant_int4_{workload}.txt") if int4 else
-                       _profile_traffic(ACT_SRC, f"act_quant_{workload}.txt"))}
+           "traffic": act_traffic}
     return roofline, act, fp4_peak
 
 

@@ -30,6 +30,28 @@ def test_profile_traffic_only_for_the_profiled_source(tmp_path, monkeypatch):
     assert bench._profile_traffic([str(src)], "k_w.txt") is None
 
 
+def test_activation_traffic_comes_from_the_kernel_that_runs(tmp_path, monkeypatch):
+    """The activation entry names the kernel the forward routes to and takes its
+    traffic from that kernel's own summary: the 128-row one at mlp_down's K,
+    the 16-row one at qkv's."""
+    (tmp_path / "profiles").mkdir()
+    s16, s128 = tmp_path / "a16.cuh", tmp_path / "a128.cuh"
+    s16.write_text("// 16-row\n")
+    s128.write_text("// 128-row\n")
+    (tmp_path / "profiles" / "act_quant_qkv.txt").write_text(
+        f"source_sha: {bench._src_sha([str(s16)])}\ntraffic_bytes_per_launch: 111\n")
+    (tmp_path / "profiles" / "act128_mlp_down.txt").write_text(
+        f"source_sha: {bench._src_sha([str(s128)])}\ntraffic_bytes_per_launch: 222\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "ACT_SRC", [str(s16)])
+    monkeypatch.setattr(bench, "A128_SRC", [str(s128)])
+    monkeypatch.setattr(bench, "_peaks", lambda: ({"hbm_gbs": 6557.4, "bf16_tflops": 1629.0}, "measured"))
+    _, act, _ = bench.kernel_rooflines(4608, 3072, 12288, 32, 0.08, 0.05, False, "mlp_down")
+    assert act["kernel"] == "act128_kernel" and act["traffic"] == 222.0
+    _, act, _ = bench.kernel_rooflines(4608, 9216, 3072, 32, 0.07, 0.02, False, "qkv")
+    assert act["kernel"] == "act_quant_kernel" and act["traffic"] == 111.0
+
+
 @pytest.mark.parametrize("fmt", ["nvfp4", "int4"])
 def test_cpu_baseline_leg(fmt):
     spec = gen.workload("small")
