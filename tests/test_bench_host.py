@@ -123,3 +123,18 @@ def test_few_token_roofline_is_one_layer_call_against_hbm():
     assert e["frac"] == pytest.approx(e["achieved"] / e["peak"], rel=1e-3)
     t = e["traffic"]
     assert t is None or t > 0
+
+
+@pytest.mark.parametrize("M,K,r,int4,kernel", [
+    (4608, 3072, 32, False, "act_quant_kernel"),      # qkv: a 128-row CTA would walk 6 stages
+    (4608, 12288, 32, False, "act128_kernel"),        # mlp_down: 24 stages per CTA at an 8-way split
+    (18432, 3072, 32, False, "act128_kernel"),        # 18432 tokens: a 2-way split, 24 stages per CTA
+    (256, 512, 32, False, "act_quant_kernel"),        # small: 8 stages in all
+    (4608, 12288, 0, False, "act_quant_kernel"),      # no rank-r branch: the 16-row kernel
+    (4608, 3072, 32, True, "act_quant_int4_kernel"),
+])
+def test_activation_kernel_name_follows_the_routing_rule(M, K, r, int4, kernel):
+    """The name bench.py reports is the kernel the forward routes to: the
+    128-row one when r > 0 and each CTA, with K split up to 8 ways at two CTAs
+    per SM, walks at least 12 stages of 64 columns."""
+    assert bench.act_kernel_name(M, K, r, int4) == kernel
